@@ -1,0 +1,108 @@
+"""Pins of the attention oracle.
+
+LoL review, 'Multi-head attention' (softmax(Q K^T / sqrt(d_k)) V per head);
+LongLive review, 'Short-Window Attention' and 'Frame Sink'."""
+import numpy as np
+import pytest
+import torch
+
+import swa_workloads as W
+from oracle import attention, rope, window
+from oracle.stream import StreamOracle
+
+
+def test_worked_example(golden):
+    g = golden("attention_small.json")
+    q = np.array(g["q"])[:, None, :]
+    k = np.array(g["k"])[:, None, :]
+    v = np.array(g["v"])[:, None, :]
+    o, lse = attention.mha(q, k, v, return_lse=True)
+    assert np.allclose(o[:, 0], g["o"], atol=1e-14)
+    assert np.allclose(lse[0], g["lse"], atol=1e-14)
+    assert np.allclose(attention.attention_probabilities(q, k)[0], g["p"], atol=1e-15)
+
+
+def test_matches_library_sdpa():
+    rng = np.random.default_rng(0)
+    q = rng.standard_normal((9, 3, 16))
+    k = rng.standard_normal((21, 3, 16))
+    v = rng.standard_normal((21, 3, 16))
+    o = attention.mha(q, k, v)
+    t = lambda a: torch.from_numpy(a).permute(1, 0, 2)[None]
+    ref = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v))[0].permute(1, 0, 2).numpy()
+    assert np.allclose(o, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_rows_sum_to_one_and_degenerate_cases():
+    rng = np.random.default_rng(1)
+    q = rng.standard_normal((5, 2, 8)) * 4
+    k = rng.standard_normal((30, 2, 8))
+    v = rng.standard_normal((30, 2, 8))
+    p = attention.attention_probabilities(q, k)
+    assert np.allclose(p.sum(-1), 1.0, atol=1e-14) and np.all(p >= 0)
+    # one key: output is that key's value
+    assert np.allclose(attention.mha(q, k[:1], v[:1]), np.broadcast_to(v[:1], q.shape), atol=1e-14)
+    # zero query: uniform weights, output = mean of V
+    assert np.allclose(attention.mha(np.zeros_like(q), k, v), np.broadcast_to(v.mean(0), q.shape), atol=1e-14)
+    # permuting the keys (with their values) changes nothing
+    perm = rng.permutation(30)
+    assert np.allclose(attention.mha(q, k[perm], v[perm]), attention.mha(q, k, v), atol=1e-13)
+
+
+def _dense_masked(qr, kr, vr, qframe_of_row, kframe_of_col, allowed, scale):
+    """Brute force: full score matrix over all frames, -inf where the key's frame
+    is not allowed for the query's frame."""
+    s = np.einsum("qhd,khd->hqk", qr, kr) * scale
+    mask = np.array([[allowed(qf, kf) for kf in kframe_of_col] for qf in qframe_of_row])
+    s = np.where(mask[None], s, -np.inf)
+    s = s - s.max(-1, keepdims=True)
+    p = np.exp(s)
+    p /= p.sum(-1, keepdims=True)
+    return np.einsum("hqk,khd->qhd", p, vr)
+
+
+@pytest.mark.parametrize("n_local,chunk", [(9, 1), (9, 3), (10_000, 1)])
+def test_stream_matches_dense_masked_brute_force(n_local, chunk):
+    """The stream oracle (history dict + A(f)) equals one dense masked softmax over
+    all frames; with a huge window it is full frame-causal attention."""
+    Wl = W.TINY
+    H, D, gh, gw = Wl.H, Wl.D, Wl.grid_h, Wl.grid_w
+    N = gh * gw
+    F = 18
+    om = rope.head_frequencies(H, Wl.pairs, 10000.0, 0.8, W.jitter_eps(5, H))
+    rng = np.random.default_rng(2)
+    Q = rng.standard_normal((F * N, H, D))
+    K = rng.standard_normal((F * N, H, D))
+    V = rng.standard_normal((F * N, H, D))
+    so = StreamOracle(H, D, gh, gw, om, Wl.pairs, t_offset=100, n_local=n_local)
+    Qr = rope.rope_frames(Q[None], 0, gh, gw, om, Wl.pairs, 100)[0]
+    Kr = rope.rope_frames(K[None], 0, gh, gw, om, Wl.pairs, 100)[0]
+    kframe = np.repeat(np.arange(F), N)
+    scale = 1 / np.sqrt(D)
+    for f0 in range(0, F, chunk):
+        so.append(f0, K[f0 * N:(f0 + chunk) * N], V[f0 * N:(f0 + chunk) * N])
+        got = so.attend(Q[f0 * N:(f0 + chunk) * N], f0)
+        last = f0 + chunk - 1
+        A = set(window.attended_frames(last, 3, n_local))
+        ref = _dense_masked(Qr[f0 * N:(f0 + chunk) * N], Kr, V, np.repeat(np.arange(f0, f0 + chunk), N),
+                            kframe, lambda qf, kf: kf in A, scale)
+        assert np.allclose(got, ref, rtol=1e-11, atol=1e-11)
+        if n_local >= F:
+            full = attention.frame_causal_attention(Qr, Kr, V, last, N)
+            if chunk == 1:
+                assert np.allclose(got, full, rtol=1e-11, atol=1e-11)
+
+
+def test_stream_rows_and_lse():
+    Wl = W.TINY
+    om = rope.head_frequencies(Wl.H, Wl.pairs, 10000.0)
+    rng = np.random.default_rng(3)
+    N = Wl.N
+    so = StreamOracle(Wl.H, Wl.D, Wl.grid_h, Wl.grid_w, om, Wl.pairs)
+    for f in range(4):
+        so.append(f, rng.standard_normal((N, Wl.H, Wl.D)), rng.standard_normal((N, Wl.H, Wl.D)))
+    q = rng.standard_normal((N, Wl.H, Wl.D))
+    full, lse = so.attend(q, 3, return_lse=True)
+    part, lse_p = so.attend(q, 3, rows=[0, 5, 23], return_lse=True)
+    assert np.allclose(part, full[[0, 5, 23]], atol=1e-14)
+    assert np.allclose(lse_p, lse[:, [0, 5, 23]], atol=1e-14)
