@@ -1,0 +1,509 @@
+"""Throughput of the sink-window attention hot path on B200.
+
+Workload (one "step"): one 40-frame prompt segment of the 240 s stream —
+30 attention layers, H=12, D=128, 1560 tokens per latent frame (30x52 grid),
+3 sink + 9 local frames, LoL jitter sigma=0.8 — in steady state: for each of
+the 40 latent frames and each of the 30 layers, RoPE + append of the frame's
+K/V into the layer's sink+ring cache, then sink-window attention of the
+frame's 1560 queries over the 12 cached frames (18720 keys). Inputs are
+seeded synthetic tensors, N(0,1)*0.5, from per-layer pools of 16 frames
+resident in HBM; the 30 caches (3.45 GB in bf16) exceed L2, so no L2 flush is
+needed between steps.
+
+Metric: latent frames/s through the 30-layer attention stack; the attention
+kernel's achieved TFLOP/s against the measured dense-bf16 peak goes in
+"roofline".
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+       [--cache bf16|fp8]
+Under torchrun each rank runs an independent replica (no collective on the
+data path; "replicas only"); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import swa_workloads as W  # noqa: E402
+
+METRIC = "latent frames/s (30-layer attn stack) + sink-window attn TFLOP/s vs B200 peak"
+UNIT = "latent frames/s"
+SEGMENT = 40          # frames per prompt segment (a KV recache every 40 frames)
+POOL = 16             # distinct input frames per layer
+
+
+def attention_flops(w: W.Workload) -> float:
+    """Algorithmic FLOPs of one layer-step of attention at steady state:
+    Q K^T and P V, 2 * Nq * Nk * D each, per head."""
+    nq = w.N * w.query_frames
+    nk = w.slots * w.N
+    return 4.0 * nq * nk * w.D * w.H
+
+
+def append_bytes(w: W.Workload, cache_elem: int) -> float:
+    """Algorithmic HBM bytes of one append: read K, V (bf16) and write them to the cache."""
+    n = w.N * w.H * w.D
+    scales = 2 * w.N * w.H * 4 if cache_elem == 1 else 0
+    return 2 * n * 2 + 2 * n * cache_elem + scales
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_index, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        # samples under load: the upper half of the clock distribution is
+        # reported as median; idle samples at the edges are dropped
+        med = statistics.median(sm) if sm else None
+        return {"sm_mhz": med, "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_index_for(local_rank: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local_rank < len(ids) and ids[local_rank].isdigit():
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+class Stream:
+    """30 layers of caches and input pools on one GPU."""
+
+    def __init__(self, w: W.Workload, cache_dtype: str, device: str, seed_offset: int = 0):
+        import sink_window_attention_b200 as swa
+        self.swa = swa
+        self.w = w
+        self.device = device
+        self.layers = w.layers
+        eps = w.eps
+        self.rope = swa.Rope(pairs=w.pairs, grid_h=w.grid_h, grid_w=w.grid_w, theta0=w.theta0, sigma_t=w.sigma_t,
+                             eps=None if eps is None else [float(e) for e in eps], t_offset=w.t_offset)
+        self.caches = [swa.KVCache(1, w.H, w.D, w.N, cache_dtype, device=device) for _ in range(self.layers)]
+        shape = (POOL, 1, w.N, w.H, w.D)
+        self.q, self.k, self.v = [], [], []
+        for l in range(self.layers):
+            base = (w.seed * 1_000_003 + (l + seed_offset) * 10_007) & ((1 << 62) - 1)
+            self.q.append(W.normal(shape, base + 1, w.qkv_scale, torch.bfloat16, device))
+            self.k.append(W.normal(shape, base + 2, w.qkv_scale, torch.bfloat16, device))
+            self.v.append(W.normal(shape, base + 3, w.qkv_scale, torch.bfloat16, device))
+        self.out = torch.empty((1, w.N, w.H, w.D), dtype=torch.bfloat16, device=device)
+        # fill every slot once so the segments below run in steady state
+        for l in range(self.layers):
+            for f in range(w.slots):
+                swa.kvcache_append(self.caches[l], self.k[l][f % POOL], self.v[l][f % POOL], f, self.rope)
+        torch.cuda.synchronize()
+
+    def step(self, seg: int, attn_events=None, qkv=None):
+        """One 40-frame segment; frames 40*(seg+1) .. 40*(seg+1)+39."""
+        swa = self.swa
+        launches = 0
+        for i in range(SEGMENT):
+            f = SEGMENT * (seg + 1) + i
+            for l in range(self.layers):
+                if qkv is None:
+                    q, k, v = self.q[l][f % POOL], self.k[l][f % POOL], self.v[l][f % POOL]
+                else:
+                    q, k, v = qkv(i, l)
+                swa.kvcache_append(self.caches[l], k, v, f, self.rope)
+                if attn_events is not None:
+                    attn_events[0].record()
+                swa.sink_window_attention(q, self.caches[l], f, self.rope, out=self.out)
+                if attn_events is not None:
+                    attn_events[1].record()
+                    attn_events[2].append((attn_events[0], attn_events[1]))
+                    attn_events[0] = torch.cuda.Event(enable_timing=True)
+                    attn_events[1] = torch.cuda.Event(enable_timing=True)
+                launches += 2
+        return launches
+
+
+def run_ours(args, rank, world, local_rank):
+    torch.cuda.set_device(local_rank)
+    from sink_window_attention_b200 import build
+    build.build()
+    import sink_window_attention_b200 as swa
+    w = W.STREAM if args.cache == "bf16" else W.STREAM_FP8
+    w = W.replace(w, layers=args.layers)
+    st = Stream(w, "bf16" if args.cache == "bf16" else "fp8", "cuda", seed_offset=1000 * rank)
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+
+    def barrier():
+        torch.cuda.synchronize()
+        if dist:
+            tdist.barrier()
+
+    for s in range(args.warmup):
+        st.step(s)
+    barrier()
+    clocks = ClockSampler(gpu_index_for(local_rank))
+    if rank == 0:
+        clocks.start()
+    ev = [torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True), []]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    t0.record()
+    launches = 0
+    for s in range(args.steps):
+        launches += st.step(args.warmup + s, attn_events=ev)
+    t1.record()
+    barrier()
+    clk = clocks.stop() if rank == 0 else None
+    ms = t0.elapsed_time(t1)
+    attn_ms = [a.elapsed_time(b) for a, b in ev[2]]
+    dev_err = swa.device_error()
+    if dev_err:
+        raise RuntimeError(f"device error word {dev_err}")
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # ---- end to end through the public API with host buffers (pinned), per step:
+    # every frame's Q/K/V of every layer is copied host -> device on a copy
+    # stream (double-buffered against compute), and each frame's last-layer
+    # output is read back.
+    e2e = run_e2e(st, args, barrier, dist)
+
+    frames = SEGMENT * args.steps * world
+    value = frames / (ms / 1e3)
+    peaks, kind = measured_peaks()
+    peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    avg_attn_s = (sum(attn_ms) / len(attn_ms)) / 1e3
+    fl = attention_flops(w)
+    achieved = fl / avg_attn_s / 1e12
+    traffic = load_traffic()
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if args.cache == "bf16" else "bf16+fp8kv",
+        "data": "synthetic",
+        "config": {"workload": f"240s stream segment: {SEGMENT} latent frames x {w.layers} layers, H=12 D=128, "
+                               f"1560 tok/frame, 3 sink + 9 local, LoL jitter 0.8, {args.cache} KV cache",
+                   "frames_per_step": SEGMENT, "layers": w.layers, "tokens_per_frame": w.N, "keys": w.slots * w.N,
+                   "heads": w.H, "head_dim": w.D, "kv_cache": args.cache, "recache": "not in the step yet",
+                   "l2": "inputs larger than L2 (30 caches x 115 MB)", "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "tensor", "kernel": "sink_window_attention_kernel",
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_kind": f"{kind} bf16 dense, sustained",
+                     "algorithmic_flops_per_launch": fl, "avg_launch_us": round(avg_attn_s * 1e6, 2)},
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+    return line
+
+
+def run_e2e(st: Stream, args, barrier, dist):
+    w = st.w
+    L = st.layers
+    n_host = 2  # host frames per layer (pinned); distinct frames cycle through them
+    host = [[tuple(t[f].cpu().pin_memory() for t in (st.q[l], st.k[l], st.v[l])) for f in range(n_host)]
+            for l in range(L)]
+    dev = [[tuple(torch.empty_like(st.q[0][0]) for _ in range(3)) for _ in range(L)] for _ in range(2)]
+    out_host = torch.empty((SEGMENT, 1, w.N, w.H, w.D), dtype=torch.bfloat16).pin_memory()
+    copy = torch.cuda.Stream()
+    comp = torch.cuda.current_stream()
+    ready = [torch.cuda.Event() for _ in range(2)]
+    free = [torch.cuda.Event() for _ in range(2)]
+    for e in free:
+        e.record(comp)
+    h2d = 3 * w.N * w.H * w.D * 2 * L * SEGMENT
+    d2h = w.N * w.H * w.D * 2 * SEGMENT
+
+    def seg(s, start=None):
+        def load(i):
+            b = i % 2
+            with torch.cuda.stream(copy):
+                if start is not None and i == 0:
+                    copy.wait_event(start)      # no copy of the timed region starts before it
+                copy.wait_event(free[b])
+                for l in range(L):
+                    for t_dev, t_host in zip(dev[b][l], host[l][(i + s) % n_host]):
+                        t_dev.copy_(t_host, non_blocking=True)
+                ready[b].record(copy)
+
+        load(0)
+        for i in range(SEGMENT):
+            if i + 1 < SEGMENT:
+                load(i + 1)
+            b = i % 2
+            comp.wait_event(ready[b])
+            f = SEGMENT * (s + 1) + i
+            for l in range(L):
+                q, k, v = dev[b][l]
+                st.swa.kvcache_append(st.caches[l], k, v, f, st.rope)
+                st.swa.sink_window_attention(q, st.caches[l], f, st.rope, out=st.out)
+            free[b].record(comp)
+            out_host[i].copy_(st.out, non_blocking=True)
+
+    steps = max(2, args.steps // 2)
+    seg(args.warmup + args.steps)
+    barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    bb = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for s in range(steps):
+        seg(args.warmup + args.steps + 1 + s, start=a if s == 0 else None)
+    bb.record()
+    barrier()
+    ms = a.elapsed_time(bb)
+    if dist:
+        import torch.distributed as tdist
+        t = torch.tensor([ms], device="cuda")
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        ms = float(t.item())
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    return {"value": round(SEGMENT * steps * world / (ms / 1e3), 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+def load_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, if any."""
+    p = os.path.join(ROOT, "profiles", "attention_traffic.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f).get("dram_bytes_per_launch")
+    return None
+
+
+# ---------------------------------------------------------------------------
+# oracle on the host cores (cpu_baseline and the --impl reference arm)
+# ---------------------------------------------------------------------------
+class OracleStep:
+    """The oracle holding a steady-state 12-frame history of one layer; each
+    call times one layer-step restricted to `rows` query rows (all heads, all
+    18720 keys) plus the K rotation of the appended frame."""
+
+    def __init__(self, w: W.Workload, seed: int = 0):
+        from oracle import rope as orope
+        from oracle.stream import StreamOracle
+        self.w = w
+        eps = w.eps
+        om = orope.head_frequencies(w.H, w.pairs, w.theta0, w.sigma_t,
+                                    None if eps is None else eps.astype(np.float64))
+        self.so = StreamOracle(w.H, w.D, w.grid_h, w.grid_w, om, w.pairs, w.t_offset)
+        self.rng = np.random.default_rng(seed)
+        self.f = 0
+        for _ in range(w.slots):
+            self._append()
+
+    def _append(self):
+        w = self.w
+        self.so.append(self.f, self.rng.standard_normal((w.N, w.H, w.D)) * w.qkv_scale,
+                       self.rng.standard_normal((w.N, w.H, w.D)) * w.qkv_scale)
+        self.f += 1
+
+    def time(self, rows: int):
+        """(seconds for the sample, seconds extrapolated to the full layer-step)."""
+        w = self.w
+        q = self.rng.standard_normal((w.N, w.H, w.D)) * w.qkv_scale
+        t0 = time.perf_counter()
+        self._append()
+        t_append = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        self.so.attend(q, self.f - 1, rows=np.arange(rows))
+        t_attn = time.perf_counter() - t0
+        return t_append + t_attn, t_append + t_attn * (w.N / rows)
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(w: W.Workload, budget_s: float = 20.0):
+    ora = OracleStep(w)
+    rows = 64
+    sample_s, full_s = ora.time(rows)
+    if sample_s < budget_s / 4:      # grow the sample towards the budget
+        rows = int(min(w.N, rows * max(1.0, (budget_s / 2) / max(sample_s, 1e-3))))
+        sample_s, full_s = ora.time(rows)
+    frames_per_s = 1.0 / (full_s * w.layers)
+    return {"value": round(frames_per_s, 6), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"one steady-state layer-step (append of 1 frame + attention of {rows} of 1560 query rows, "
+                      f"all 12 heads, 18720 keys) in float64 NumPy; took {sample_s:.2f} s; extrapolated to the "
+                      f"full layer-step ({full_s:.2f} s) and to {w.layers} layers"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    w = W.STREAM
+    rows = 128
+    ora = OracleStep(w)
+    samples = []
+    for s in range(args.warmup + args.steps):
+        _, full_s = ora.time(rows)
+        if s >= args.warmup:
+            samples.append(full_s)
+    per_frame = statistics.mean(samples) * w.layers
+    value = 1.0 / per_frame
+    sample = (f"each step: the oracle (float64 NumPy) on one steady-state layer-step, {rows} of 1560 query rows, "
+              f"extrapolated to the full layer-step and {w.layers} layers")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_frame * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"240s stream segment: latent frames x {w.layers} layers, H=12 D=128, "
+                                   "1560 tok/frame, 3 sink + 9 local, LoL jitter 0.8",
+                       "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def run_attention_only(args):
+    """Wan-shaped single layer (H=12, D=128, 1560 queries over 18720 keys):
+    `warmup` + `steps` attention launches at steady state, each timed with CUDA
+    events on the launching stream. A small, self-contained case for kernel
+    timing and profiler captures."""
+    from sink_window_attention_b200 import build
+    build.build()
+    import sink_window_attention_b200 as swa
+    w = W.WAN if args.workload == "wan" else W.CHUNK
+    st = Stream(W.replace(w, layers=1, sigma_t=0.8, jitter_seed=4), "bf16", "cuda")
+    c = w.query_frames
+    q = W.normal((1, c * w.N, w.H, w.D), 99, w.qkv_scale, torch.bfloat16, "cuda")
+    out = torch.empty_like(q)
+    f0 = 3 * 40  # a steady-state frame (chunk start) with all 12 slots valid
+    times = []
+    for i in range(args.warmup + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        swa.sink_window_attention(q, st.caches[0], f0, st.rope, out=out)
+        b.record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(a.elapsed_time(b) / 1e3)
+    assert swa.device_error() == 0
+    fl = 4.0 * (c * w.N) * (w.slots * w.N) * w.D * w.H
+    peaks, kind = measured_peaks()
+    t = statistics.median(times)
+    return {"mode": "attention", "workload": w.name, "launches": len(times), "median_us": round(t * 1e6, 2),
+            "min_us": round(min(times) * 1e6, 2), "tflops": round(fl / t / 1e12, 1),
+            "frac_of_burst_peak": round(fl / t / 1e12 / peaks["bf16_tflops"], 4), "peak_kind": kind}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=8)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cache", default="bf16", choices=["bf16", "fp8"])
+    ap.add_argument("--layers", type=int, default=30)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--mode", default="stream", choices=["stream", "attention"])
+    ap.add_argument("--workload", default="wan", choices=["wan", "chunk"])
+    args = ap.parse_args()
+    if args.mode == "attention":
+        print(json.dumps(run_attention_only(args)), flush=True)
+        return
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as tdist
+            tdist.barrier()
+            tdist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

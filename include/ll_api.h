@@ -1,0 +1,205 @@
+/*
+ * ll_api.h — C ABI of the B200 sink-window attention library (libll_swa.so).
+ *
+ * The method (LongLive: Real-time Interactive Long Video Generation, paper
+ * review; LoL: Longer than Longer, paper review) generates video latent frame
+ * by latent frame. Every new frame (or 3-frame chunk) attends, per head, to
+ * the KV of 3 pinned "frame sink" frames plus a short window of the most
+ * recent frames (LongLive review, sections "Short-Window Attention" and
+ * "Frame Sink": 9 local + 3 sink = 12 effective frames). Q and K carry a
+ * factorised 3D rotary embedding whose temporal base frequency is jittered per
+ * head (LoL review, "Method steps"). At a prompt switch the cached frames' K/V
+ * are recomputed (LongLive review, "KV Recache").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensor pointers are DEVICE pointers into caller-owned memory unless a
+ *   parameter says "host". The library never allocates device memory and keeps
+ *   no state between calls; every call is asynchronous on `stream`
+ *   (a cudaStream_t passed as void*, NULL = legacy default stream).
+ * - Token tensors use the layout [B][T][H][D] (row-major, D fastest), with
+ *   T = frames * N, N = grid_h * grid_w tokens per latent frame in row-major
+ *   (grid row, grid column) order.
+ * - The KV cache of one layer is [B][S*N][H][D], S = n_sink + n_local slots of
+ *   N tokens each (slot s holds tokens [s*N, (s+1)*N)). Frame f is stored in
+ *   slot f when f < n_sink and in slot n_sink + (f - n_sink) mod n_local
+ *   otherwise. After frames 0..f have been written, the occupied slots are the
+ *   prefix [0, min(f+1, S)) and they hold exactly the frames a query at frame f
+ *   attends to.
+ * - Arguments are validated on the host before anything is launched; a bad
+ *   argument returns LL_ERR_INVALID_ARG and ll_last_error() says why.
+ *   LL_ERR_UNSUPPORTED marks a well-formed request this build does not
+ *   implement. LL_ERR_CUDA reports a failed launch or runtime call.
+ * - Device-side waits are bounded. A wait that gives up records a code in the
+ *   library's device error word and the kernel returns early (its outputs are
+ *   then undefined); ll_device_error() reads and clears that word.
+ */
+#ifndef LL_API_H
+#define LL_API_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LL_ABI_VERSION 1
+#define LL_MAX_HEADS 64
+
+typedef enum ll_status {
+  LL_OK = 0,
+  LL_ERR_INVALID_ARG = 1,
+  LL_ERR_UNSUPPORTED = 2,
+  LL_ERR_CUDA = 3,
+  LL_ERR_TIMEOUT = 4
+} ll_status;
+
+typedef enum ll_dtype {
+  LL_F32 = 0,       /* IEEE float32 */
+  LL_BF16 = 1,      /* bfloat16 */
+  LL_FP8_E4M3 = 2   /* OCP E4M3 with one fp32 scale per (token, head); cache storage only */
+} ll_dtype;
+
+/*
+ * Factorised 3D rotary embedding with LoL per-head jitter.
+ * LoL review, "Prerequisites: RoPE": a channel pair (x_{2j}, x_{2j+1}) at
+ * position p is rotated by [[cos p*w, -sin p*w], [sin p*w, cos p*w]] with
+ * w_i = base^(-2i/d). LoL review, "Method steps": theta_hat_h =
+ * theta0 * (1 + sigma * eps_h) is the base of head h.
+ * Layout: the D/2 pairs of a head are a temporal band of pairs_t pairs, then
+ * pairs_h pairs for the grid row and pairs_w for the grid column; inside a
+ * band of P pairs, i = 0..P-1 and d = 2P. The temporal band of head h uses
+ * base theta0 * (1 + sigma_t * eps_h[h]); the two spatial bands use theta0.
+ * Token (frame f, row r, column c) sits at position (t_offset + f, r, c).
+ */
+typedef struct ll_rope_desc {
+  int pairs_t, pairs_h, pairs_w;  /* pairs per axis; pairs_t + pairs_h + pairs_w = D/2 */
+  double theta0;                  /* base frequency, > 1 */
+  double sigma_t;                 /* jitter scale on the temporal band, 0 <= sigma_t < 1 */
+  const float* eps_h;             /* HOST pointer to H draws in [-1, 1], or NULL for no jitter */
+  int grid_h, grid_w;             /* token grid of one latent frame */
+  long long t_offset;             /* temporal position of frame 0 */
+} ll_rope_desc;
+
+/*
+ * One layer's sink + ring KV cache (caller-owned device memory).
+ * k, v: [B][S*N][H][D] of `dtype` (F32, BF16 or FP8_E4M3).
+ * k_scale, v_scale: [B][S*N][H] fp32 dequantisation scales, FP8 only
+ * (value = decode(code) * scale); NULL for the other dtypes.
+ */
+typedef struct ll_kvcache {
+  void* k;
+  void* v;
+  float* k_scale;
+  float* v_scale;
+  ll_dtype dtype;
+  int B, H, D;
+  int tokens_per_frame;   /* N; must equal rope grid_h * grid_w when a rope desc is given */
+  int n_sink, n_local;    /* 3 and 9 in the pages' setting */
+} ll_kvcache;
+
+/* ABI version of the loaded library (LL_ABI_VERSION at build time). */
+int ll_abi_version(void);
+
+/* Message describing the last failure on the calling thread ("" if none). */
+const char* ll_last_error(void);
+
+/*
+ * Slot of frame `frame` in a cache with n_sink pinned and n_local ring slots.
+ * Host only (no GPU needed). LongLive review, "Frame Sink": the sink frames
+ * are pinned; the short window keeps the most recent local frames.
+ * Errors: LL_ERR_INVALID_ARG for frame < 0, n_sink < 0, n_local < 1 or slot NULL.
+ */
+ll_status ll_slot_of_frame(long long frame, int n_sink, int n_local, int* slot);
+
+/*
+ * Synchronises `stream`, then copies the device error word into *code
+ * (0 = no error; bit 0 = a bounded wait gave up) and clears it.
+ * Returns LL_ERR_TIMEOUT when the word was non-zero.
+ */
+ll_status ll_device_error(int* code, void* stream);
+
+/*
+ * In-place 3D RoPE of x [B][n_frames*N][H][D] (dtype F32 or BF16) holding the
+ * consecutive frames first_frame .. first_frame + n_frames - 1.
+ * LoL review, "Method steps" (6): (Q'_h, K'_h) = RoPERotate(Q_h, K_h, omega_h).
+ * Errors: LL_ERR_INVALID_ARG for NULL x or rope, non-positive sizes,
+ * first_frame < 0, D odd or pairs not summing to D/2, H > LL_MAX_HEADS.
+ */
+ll_status ll_rope_apply(void* x, ll_dtype dtype, int B, int n_frames, int H, int D,
+                        long long first_frame, const ll_rope_desc* rope, void* stream);
+
+/*
+ * Append frames first_frame .. first_frame + n_frames - 1 to the cache.
+ * k, v: [B][n_frames*N][H][D] of in_dtype (F32 or BF16; BF16 for an FP8 cache).
+ * K is rotated with `rope` at each frame's own position before it is stored
+ * (rope NULL: k is stored as given). Frame f overwrites slot(f), which evicts
+ * the oldest local frame once the ring is full (LongLive review, "Frame Sink"
+ * and "Short-Window Attention"). For an FP8 cache each (token, head) row is
+ * stored as E4M3 codes of x / scale with scale = max|x| / 448 (1 for a zero
+ * row), round-to-nearest-even with saturation.
+ * slots_out: optional HOST array of n_frames ints receiving the slots written.
+ * Errors: LL_ERR_INVALID_ARG for NULL tensors, first_frame < 0,
+ * n_frames < 1 or > n_local (a call may not overwrite its own frames),
+ * dtype mismatch with the cache, rope grid inconsistent with N.
+ */
+ll_status ll_kvcache_append(const ll_kvcache* cache, const void* k, const void* v,
+                            ll_dtype in_dtype, long long first_frame, int n_frames,
+                            const ll_rope_desc* rope, int* slots_out, void* stream);
+
+/*
+ * Attention of the query frames first_frame .. first_frame + n_query_frames - 1
+ * over every cached token of the frames they may see: with f the last query
+ * frame, the key set is all tokens of slots [0, min(f+1, S)), i.e. the 3 sink
+ * frames plus the most recent frames up to f (LongLive review,
+ * "Short-Window Attention", "Frame Sink"). The query frames must already be
+ * in the cache (append first). Inside the key set there is no mask, so the
+ * tokens of a query frame or chunk see each other (frame-level causality).
+ * Per head h: out = softmax(Q'_h K_h^T * softmax_scale) V_h
+ * (LoL review, "Multi-head attention"), with Q' = RoPE(Q) when rope != NULL
+ * (rope NULL: q is already rotated).
+ * q, out: [B][n_query_frames*N][H][D]; BF16 for BF16 and FP8 caches, F32 for an
+ * F32 cache. softmax_scale 0 means 1/sqrt(D). lse (optional, NULL to skip):
+ * [B][H][n_query_frames*N] fp32 natural-log sum of exp of the scaled scores.
+ * workspace: device scratch of at least
+ * ll_sink_window_attention_workspace_bytes(...) bytes (NULL allowed when that
+ * is 0); its contents need not be initialised and are clobbered.
+ * Errors: LL_ERR_INVALID_ARG for NULL tensors, first_frame < 0,
+ * n_query_frames < 1 or > n_local, a workspace that is too small;
+ * LL_ERR_UNSUPPORTED for D other than 64 or 128.
+ */
+size_t ll_sink_window_attention_workspace_bytes(const ll_kvcache* cache, int n_query_frames);
+
+ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvcache* cache,
+                                   long long first_frame, int n_query_frames,
+                                   const ll_rope_desc* rope, float softmax_scale,
+                                   void* out, float* lse, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/*
+ * KV recache at a prompt switch (LongLive review, "KV Recache": the cache is
+ * rebuilt from the generated frames together with the new prompt).
+ * Slots 0..n_slots-1 are recomputed from hidden states x [B][n_slots*N][d_model]
+ * (BF16; rows of slot s belong to the frame held in slot s):
+ *   K = RoPE(RMSNorm(x Wk; gamma, rms_eps)),  V = x Wv,
+ * RMSNorm over the whole H*D-wide row, RoPE at each slot's frame position.
+ * wk, wv: [d_model][H*D] BF16 row-major; gamma: [H*D] fp32.
+ * slot_frames: HOST array of n_slots absolute frame indices (frame in slot s).
+ * workspace: device scratch of at least ll_kv_recache_workspace_bytes(...)
+ * bytes. The cache may be BF16 or FP8.
+ * Errors: LL_ERR_INVALID_ARG for NULL pointers, n_slots outside [1, S],
+ * negative frames; LL_ERR_UNSUPPORTED for d_model or H*D not a multiple of 128.
+ */
+size_t ll_kv_recache_workspace_bytes(const ll_kvcache* cache, int d_model, int n_slots);
+
+ll_status ll_kv_recache(const ll_kvcache* cache, const void* x, int d_model,
+                        const void* wk, const void* wv, const float* gamma, float rms_eps,
+                        const long long* slot_frames, int n_slots, const ll_rope_desc* rope,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LL_API_H */

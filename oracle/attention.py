@@ -40,9 +40,10 @@ def mha(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float | None = None,
     D = q.shape[-1]
     if scale is None:
         scale = 1.0 / np.sqrt(D)
-    s = np.einsum("qhd,khd->hqk", q, k) * scale          # [H, Tq, Tk]
+    # per-head score matrix Q_h K_h^T (matmul over [H, Tq, D] x [H, D, Tk])
+    s = np.matmul(q.transpose(1, 0, 2), k.transpose(1, 2, 0)) * scale   # [H, Tq, Tk]
     p = softmax_rows(s)
-    o = np.einsum("hqk,khd->qhd", p, v)
+    o = np.matmul(p, v.transpose(1, 0, 2)).transpose(1, 0, 2)           # [Tq, H, D]
     if not return_lse:
         return o
     m = np.max(s, axis=-1)

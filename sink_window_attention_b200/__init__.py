@@ -1,0 +1,245 @@
+"""Python binding of libll_swa.so (the B200 sink-window attention library).
+
+Argument marshalling only: torch tensors supply device memory and the CUDA
+stream; every step of the computation runs in the library's CUDA kernels.
+The shared library must have been built (``python -m
+sink_window_attention_b200.build`` or ``__graft_entry__.build()``); importing
+this package without it raises, there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libll_swa.so")
+
+LL_OK, LL_ERR_INVALID_ARG, LL_ERR_UNSUPPORTED, LL_ERR_CUDA, LL_ERR_TIMEOUT = range(5)
+LL_F32, LL_BF16, LL_FP8_E4M3 = 0, 1, 2
+MAX_HEADS = 64
+
+EXPORTED = (
+    "ll_abi_version", "ll_last_error", "ll_slot_of_frame", "ll_device_error", "ll_rope_apply",
+    "ll_kvcache_append", "ll_sink_window_attention_workspace_bytes", "ll_sink_window_attention",
+    "ll_kv_recache_workspace_bytes", "ll_kv_recache",
+)
+
+
+class LLError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"ll status {status}: {message}")
+        self.status = status
+
+
+class RopeDescC(ctypes.Structure):
+    _fields_ = [("pairs_t", ctypes.c_int), ("pairs_h", ctypes.c_int), ("pairs_w", ctypes.c_int),
+                ("theta0", ctypes.c_double), ("sigma_t", ctypes.c_double),
+                ("eps_h", ctypes.POINTER(ctypes.c_float)), ("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int),
+                ("t_offset", ctypes.c_longlong)]
+
+
+class KVCacheC(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("k_scale", ctypes.c_void_p),
+                ("v_scale", ctypes.c_void_p), ("dtype", ctypes.c_int), ("B", ctypes.c_int), ("H", ctypes.c_int),
+                ("D", ctypes.c_int), ("tokens_per_frame", ctypes.c_int), ("n_sink", ctypes.c_int),
+                ("n_local", ctypes.c_int)]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with sink_window_attention_b200.build.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, ll_, f, d, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float, ctypes.c_double, ctypes.c_size_t
+        rp, cp = ctypes.POINTER(RopeDescC), ctypes.POINTER(KVCacheC)
+        L.ll_abi_version.restype = i
+        L.ll_last_error.restype = ctypes.c_char_p
+        L.ll_slot_of_frame.argtypes = [ll_, i, i, ctypes.POINTER(i)]
+        L.ll_device_error.argtypes = [ctypes.POINTER(i), vp]
+        L.ll_rope_apply.argtypes = [vp, i, i, i, i, i, ll_, rp, vp]
+        L.ll_kvcache_append.argtypes = [cp, vp, vp, i, ll_, i, rp, ctypes.POINTER(i), vp]
+        L.ll_sink_window_attention_workspace_bytes.argtypes = [cp, i]
+        L.ll_sink_window_attention_workspace_bytes.restype = sz
+        L.ll_sink_window_attention.argtypes = [vp, i, cp, ll_, i, rp, f, vp, vp, vp, sz, vp]
+        L.ll_kv_recache_workspace_bytes.argtypes = [cp, i, i]
+        L.ll_kv_recache_workspace_bytes.restype = sz
+        L.ll_kv_recache.argtypes = [cp, vp, i, vp, vp, vp, f, ctypes.POINTER(ll_), i, rp, vp, sz, vp]
+        for name in EXPORTED[2:]:
+            if name not in ("ll_sink_window_attention_workspace_bytes", "ll_kv_recache_workspace_bytes"):
+                getattr(L, name).restype = i
+        _lib = L
+    return _lib
+
+
+def last_error() -> str:
+    return lib().ll_last_error().decode()
+
+
+def _check(status: int) -> None:
+    if status != LL_OK:
+        raise LLError(status, last_error())
+
+
+def _stream(stream=None) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    if t == torch.float32:
+        return LL_F32
+    if t == torch.bfloat16:
+        return LL_BF16
+    raise ValueError(f"unsupported tensor dtype {t}")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+@dataclass
+class Rope:
+    """3D RoPE with the LoL per-head jittered temporal base (mirrors ll_rope_desc)."""
+    pairs: Sequence[int]
+    grid_h: int
+    grid_w: int
+    theta0: float = 10000.0
+    sigma_t: float = 0.0
+    eps: Optional[Sequence[float]] = None
+    t_offset: int = 0
+
+    def to_c(self) -> RopeDescC:
+        r = RopeDescC()
+        r.pairs_t, r.pairs_h, r.pairs_w = (int(x) for x in self.pairs)
+        r.theta0 = float(self.theta0)
+        r.sigma_t = float(self.sigma_t)
+        if self.eps is not None:
+            arr = (ctypes.c_float * len(self.eps))(*[float(e) for e in self.eps])
+            r._eps_keepalive = arr  # noqa: keep the host array alive with the struct
+            r.eps_h = ctypes.cast(arr, ctypes.POINTER(ctypes.c_float))
+        r.grid_h, r.grid_w, r.t_offset = int(self.grid_h), int(self.grid_w), int(self.t_offset)
+        return r
+
+
+def _rope_ref(rope: Optional[Rope]):
+    return ctypes.byref(rope.to_c()) if rope is not None else None
+
+
+class KVCache:
+    """One layer's sink + ring KV cache in device memory (mirrors ll_kvcache)."""
+
+    def __init__(self, B: int, H: int, D: int, tokens_per_frame: int, dtype: str = "bf16",
+                 n_sink: int = 3, n_local: int = 9, device: str = "cuda"):
+        self.B, self.H, self.D, self.N = B, H, D, tokens_per_frame
+        self.n_sink, self.n_local = n_sink, n_local
+        self.S = n_sink + n_local
+        self.dtype = dtype
+        shape = (B, self.S * tokens_per_frame, H, D)
+        if dtype == "fp8":
+            self.k = torch.zeros(shape, dtype=torch.uint8, device=device)
+            self.v = torch.zeros(shape, dtype=torch.uint8, device=device)
+            self.k_scale = torch.ones(shape[:3], dtype=torch.float32, device=device)
+            self.v_scale = torch.ones(shape[:3], dtype=torch.float32, device=device)
+            self.code = LL_FP8_E4M3
+        else:
+            tdt = {"bf16": torch.bfloat16, "f32": torch.float32}[dtype]
+            self.k = torch.zeros(shape, dtype=tdt, device=device)
+            self.v = torch.zeros(shape, dtype=tdt, device=device)
+            self.k_scale = self.v_scale = None
+            self.code = _dtype_code(tdt)
+
+    def to_c(self) -> KVCacheC:
+        c = KVCacheC()
+        c.k, c.v = self.k.data_ptr(), self.v.data_ptr()
+        c.k_scale = self.k_scale.data_ptr() if self.k_scale is not None else None
+        c.v_scale = self.v_scale.data_ptr() if self.v_scale is not None else None
+        c.dtype, c.B, c.H, c.D = self.code, self.B, self.H, self.D
+        c.tokens_per_frame, c.n_sink, c.n_local = self.N, self.n_sink, self.n_local
+        return c
+
+
+def abi_version() -> int:
+    return lib().ll_abi_version()
+
+
+def slot_of_frame(frame: int, n_sink: int = 3, n_local: int = 9) -> int:
+    s = ctypes.c_int(-1)
+    _check(lib().ll_slot_of_frame(frame, n_sink, n_local, ctypes.byref(s)))
+    return s.value
+
+
+def device_error(stream=None) -> int:
+    """Synchronise and read (then clear) the library's device error word."""
+    code = ctypes.c_int(0)
+    st = lib().ll_device_error(ctypes.byref(code), _stream(stream))
+    if st not in (LL_OK, LL_ERR_TIMEOUT):
+        _check(st)
+    return code.value
+
+
+def rope_apply(x: torch.Tensor, first_frame: int, rope: Rope, stream=None) -> torch.Tensor:
+    """In-place 3D RoPE of x [B, F*N, H, D]."""
+    B, T, H, D = x.shape
+    N = rope.grid_h * rope.grid_w
+    _check(lib().ll_rope_apply(_ptr(x), _dtype_code(x.dtype), B, T // N, H, D, first_frame, _rope_ref(rope),
+                               _stream(stream)))
+    return x
+
+
+def kvcache_append(cache: KVCache, k: torch.Tensor, v: torch.Tensor, first_frame: int,
+                   rope: Optional[Rope], stream=None):
+    """Write frames first_frame.. of k, v [B, F*N, H, D] into their slots; returns the slots."""
+    F = k.shape[1] // cache.N
+    slots = (ctypes.c_int * F)()
+    _check(lib().ll_kvcache_append(ctypes.byref(cache.to_c()), _ptr(k), _ptr(v), _dtype_code(k.dtype), first_frame,
+                                   F, _rope_ref(rope), slots, _stream(stream)))
+    return list(slots)
+
+
+def attention_workspace_bytes(cache: KVCache, n_query_frames: int) -> int:
+    return int(lib().ll_sink_window_attention_workspace_bytes(ctypes.byref(cache.to_c()), n_query_frames))
+
+
+def sink_window_attention(q: torch.Tensor, cache: KVCache, first_frame: int, rope: Optional[Rope],
+                          softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                          lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                          stream=None) -> torch.Tensor:
+    """Attention of query frames first_frame.. (q [B, F*N, H, D]) over the cache."""
+    F = q.shape[1] // cache.N
+    if out is None:
+        out = torch.empty_like(q)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().ll_sink_window_attention(_ptr(q), _dtype_code(q.dtype), ctypes.byref(cache.to_c()), first_frame, F,
+                                          _rope_ref(rope), float(softmax_scale), _ptr(out), _ptr(lse),
+                                          _ptr(workspace), ws_bytes, _stream(stream)))
+    return out
+
+
+def recache_workspace_bytes(cache: KVCache, d_model: int, n_slots: int) -> int:
+    return int(lib().ll_kv_recache_workspace_bytes(ctypes.byref(cache.to_c()), d_model, n_slots))
+
+
+def kv_recache(cache: KVCache, x: torch.Tensor, wk: torch.Tensor, wv: torch.Tensor, gamma: torch.Tensor,
+               rms_eps: float, slot_frames: Sequence[int], rope: Rope,
+               workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Recompute K/V of slots 0..len(slot_frames)-1 from hidden states x [B, n*N, d_model]."""
+    n = len(slot_frames)
+    frames = (ctypes.c_longlong * n)(*[int(f) for f in slot_frames])
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().ll_kv_recache(ctypes.byref(cache.to_c()), _ptr(x), x.shape[-1], _ptr(wk), _ptr(wv), _ptr(gamma),
+                               float(rms_eps), frames, n, _rope_ref(rope), _ptr(workspace), ws_bytes,
+                               _stream(stream)))

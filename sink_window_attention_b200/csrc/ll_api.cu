@@ -1,0 +1,342 @@
+// ll_api.cu — host side of libll_swa.so: argument validation, TMA tensor-map
+// encoding and kernel launches behind the C ABI declared in include/ll_api.h.
+// The library allocates no device memory and keeps no state between calls.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "../../include/ll_api.h"
+#include "ll_attention.cuh"
+#include "ll_common.cuh"
+#include "ll_rope_append.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+ll_status fail(ll_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+ll_status check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(LL_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return LL_OK;
+}
+
+int element_size(ll_dtype t) {
+  switch (t) {
+    case LL_F32: return 4;
+    case LL_BF16: return 2;
+    case LL_FP8_E4M3: return 1;
+  }
+  return 0;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Validates a rope descriptor for heads H and head dim D and converts it.
+ll_status make_rope(const ll_rope_desc* r, int H, int D, long long t_first, ll::RopeParams* out) {
+  std::memset(out, 0, sizeof(*out));
+  if (r == nullptr) return LL_OK;  // disabled
+  if (r->pairs_t < 0 || r->pairs_h < 0 || r->pairs_w < 0 || r->pairs_t + r->pairs_h + r->pairs_w != D / 2)
+    return fail(LL_ERR_INVALID_ARG, "rope pairs (%d, %d, %d) must be >= 0 and sum to D/2 = %d", r->pairs_t,
+                r->pairs_h, r->pairs_w, D / 2);
+  if (!(r->theta0 > 1.0) || !std::isfinite(r->theta0))
+    return fail(LL_ERR_INVALID_ARG, "rope theta0 must be a finite value > 1");
+  if (!(r->sigma_t >= 0.0 && r->sigma_t < 1.0))
+    return fail(LL_ERR_INVALID_ARG, "rope sigma_t must lie in [0, 1) so every base stays positive");
+  if (r->grid_h < 1 || r->grid_w < 1) return fail(LL_ERR_INVALID_ARG, "rope grid must be at least 1x1");
+  if (H > ll::kMaxHeads) return fail(LL_ERR_INVALID_ARG, "H = %d exceeds %d", H, ll::kMaxHeads);
+  if (r->t_offset < 0) return fail(LL_ERR_INVALID_ARG, "rope t_offset must be >= 0");
+  out->enabled = 1;
+  out->pt = r->pairs_t;
+  out->ph = r->pairs_h;
+  out->pw = r->pairs_w;
+  out->grid_w = r->grid_w;
+  out->t_first = r->t_offset + t_first;
+  out->theta0 = r->theta0;
+  out->sigma = r->eps_h ? r->sigma_t : 0.0;
+  for (int h = 0; h < H; ++h) {
+    const float e = r->eps_h ? r->eps_h[h] : 0.f;
+    if (!(e >= -1.f && e <= 1.f)) return fail(LL_ERR_INVALID_ARG, "eps_h[%d] = %g is outside [-1, 1]", h, e);
+    out->eps[h] = e;
+  }
+  return LL_OK;
+}
+
+ll_status check_cache(const ll_kvcache* c) {
+  if (c == nullptr) return fail(LL_ERR_INVALID_ARG, "cache is NULL");
+  if (c->k == nullptr || c->v == nullptr) return fail(LL_ERR_INVALID_ARG, "cache k/v pointer is NULL");
+  if (!aligned16(c->k) || !aligned16(c->v)) return fail(LL_ERR_INVALID_ARG, "cache k/v must be 16-byte aligned");
+  if (element_size(c->dtype) == 0) return fail(LL_ERR_INVALID_ARG, "unknown cache dtype %d", (int)c->dtype);
+  if (c->dtype == LL_FP8_E4M3 && (c->k_scale == nullptr || c->v_scale == nullptr))
+    return fail(LL_ERR_INVALID_ARG, "an FP8 cache needs k_scale and v_scale");
+  if (c->B < 1 || c->H < 1 || c->D < 2 || c->tokens_per_frame < 1)
+    return fail(LL_ERR_INVALID_ARG, "cache sizes must be positive (B=%d H=%d D=%d N=%d)", c->B, c->H, c->D,
+                c->tokens_per_frame);
+  if (c->D % 16 != 0) return fail(LL_ERR_INVALID_ARG, "D = %d must be a multiple of 16", c->D);
+  if (c->H > ll::kMaxHeads) return fail(LL_ERR_INVALID_ARG, "H = %d exceeds %d", c->H, ll::kMaxHeads);
+  if (c->n_sink < 0 || c->n_local < 1) return fail(LL_ERR_INVALID_ARG, "need n_sink >= 0 and n_local >= 1");
+  return LL_OK;
+}
+
+ll_status check_grid(const ll_rope_desc* r, int N) {
+  if (r && r->grid_h * r->grid_w != N)
+    return fail(LL_ERR_INVALID_ARG, "rope grid %dx%d does not match %d tokens per frame", r->grid_h, r->grid_w, N);
+  return LL_OK;
+}
+
+int num_sms() {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  return sms;
+}
+
+// ---------------------------------------------------------------------------
+// TMA tensor maps (driver entry point fetched through the runtime, so the
+// library does not link libcuda directly).
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 4D map over a [B][rows][H][D] tensor whose batch stride is batch_rows rows:
+// dims (D, H, rows, B), box (128 bytes of D, 1 head, box_rows, 1), 128-byte
+// swizzle, rows >= `rows` read as zeros.
+ll_status encode_rows_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int es, int D, int H,
+                          long long rows, long long batch_rows, int B, int box_rows,
+                          CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(LL_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)D * es, (cuuint64_t)H * D * es, (cuuint64_t)batch_rows * H * D * es};
+  const cuuint32_t box[4] = {(cuuint32_t)(128 / es), 1u, (cuuint32_t)box_rows, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  const CUresult r = fn(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LL_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return LL_OK;
+}
+
+template <class TR>
+ll_status launch_attention(const ll::AttnParams& p, const ll_kvcache* c, long long S, cudaStream_t stream) {
+  CUtensorMap tmK, tmV;
+  const CUtensorMapDataType dt = TR::ES == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const long long batch_rows = S * c->tokens_per_frame;
+  ll_status st = encode_rows_map(&tmK, c->k, dt, TR::ES, TR::D, c->H, p.Nk, batch_rows, c->B, TR::BN);
+  if (st != LL_OK) return st;
+  st = encode_rows_map(&tmV, c->v, dt, TR::ES, TR::D, c->H, p.Nk, batch_rows, c->B, TR::BN,
+                       TR::ES == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B);
+  if (st != LL_OK) return st;
+  auto kern = ll::sink_window_attention_kernel<TR>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TR::SMEM_BYTES) != cudaSuccess)
+      return check_launch("cudaFuncSetAttribute(attention)");
+    attr_set = true;
+  }
+  const dim3 grid((p.Tq + TR::BM - 1) / TR::BM, c->H, c->B);
+  kern<<<grid, TR::THREADS, TR::SMEM_BYTES, stream>>>(tmK, tmV, p);
+  return check_launch("sink_window_attention_kernel");
+}
+
+}  // namespace
+
+extern "C" {
+
+int ll_abi_version(void) { return LL_ABI_VERSION; }
+
+const char* ll_last_error(void) { return g_last_error.c_str(); }
+
+ll_status ll_slot_of_frame(long long frame, int n_sink, int n_local, int* slot) {
+  if (slot == nullptr) return fail(LL_ERR_INVALID_ARG, "slot is NULL");
+  if (frame < 0 || n_sink < 0 || n_local < 1)
+    return fail(LL_ERR_INVALID_ARG, "need frame >= 0, n_sink >= 0, n_local >= 1");
+  *slot = frame < n_sink ? static_cast<int>(frame) : n_sink + static_cast<int>((frame - n_sink) % n_local);
+  return LL_OK;
+}
+
+ll_status ll_device_error(int* code, void* stream) {
+  if (code == nullptr) return fail(LL_ERR_INVALID_ARG, "code is NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return check_launch("cudaStreamSynchronize");
+  unsigned int w = 0;
+  if (cudaMemcpyFromSymbol(&w, ll::g_error_word, sizeof(w)) != cudaSuccess) return check_launch("read error word");
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(ll::g_error_word, &zero, sizeof(zero)) != cudaSuccess)
+    return check_launch("clear error word");
+  *code = static_cast<int>(w);
+  if (w != 0) return fail(LL_ERR_TIMEOUT, "a device-side wait gave up (error word 0x%x)", w);
+  return LL_OK;
+}
+
+ll_status ll_rope_apply(void* x, ll_dtype dtype, int B, int n_frames, int H, int D, long long first_frame,
+                        const ll_rope_desc* rope, void* stream) {
+  g_last_error.clear();
+  if (x == nullptr || rope == nullptr) return fail(LL_ERR_INVALID_ARG, "x and rope must be non-NULL");
+  if (!aligned16(x)) return fail(LL_ERR_INVALID_ARG, "x must be 16-byte aligned");
+  if (B < 1 || n_frames < 1 || H < 1 || D < 2) return fail(LL_ERR_INVALID_ARG, "sizes must be positive");
+  if (D % 8 != 0) return fail(LL_ERR_INVALID_ARG, "D = %d must be a multiple of 8", D);
+  if (first_frame < 0) return fail(LL_ERR_INVALID_ARG, "first_frame must be >= 0");
+  if (dtype != LL_F32 && dtype != LL_BF16) return fail(LL_ERR_INVALID_ARG, "rope_apply takes F32 or BF16");
+  ll::RopeApplyParams p{};
+  ll_status st = make_rope(rope, H, D, first_frame, &p.rp);
+  if (st != LL_OK) return st;
+  p.x = x;
+  p.B = B;
+  p.F = n_frames;
+  p.N = rope->grid_h * rope->grid_w;
+  p.H = H;
+  p.D = D;
+  const long long chunks = static_cast<long long>(B) * n_frames * p.N * H * (D / 8);
+  const long long want = (chunks + 255) / 256;
+  const int grid = static_cast<int>(want < 8LL * num_sms() ? want : 8LL * num_sms());
+  const size_t smem = static_cast<size_t>(H) * (D / 2) * sizeof(float);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == LL_BF16)
+    ll::rope_apply_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(p);
+  else
+    ll::rope_apply_kernel<float><<<grid, 256, smem, s>>>(p);
+  return check_launch("rope_apply_kernel");
+}
+
+ll_status ll_kvcache_append(const ll_kvcache* cache, const void* k, const void* v, ll_dtype in_dtype,
+                            long long first_frame, int n_frames, const ll_rope_desc* rope, int* slots_out,
+                            void* stream) {
+  g_last_error.clear();
+  ll_status st = check_cache(cache);
+  if (st != LL_OK) return st;
+  if (k == nullptr || v == nullptr) return fail(LL_ERR_INVALID_ARG, "k and v must be non-NULL");
+  if (!aligned16(k) || !aligned16(v)) return fail(LL_ERR_INVALID_ARG, "k and v must be 16-byte aligned");
+  if (first_frame < 0) return fail(LL_ERR_INVALID_ARG, "first_frame must be >= 0");
+  if (n_frames < 1 || n_frames > cache->n_local)
+    return fail(LL_ERR_INVALID_ARG, "n_frames = %d must lie in [1, n_local = %d]", n_frames, cache->n_local);
+  if (in_dtype != LL_F32 && in_dtype != LL_BF16) return fail(LL_ERR_INVALID_ARG, "k/v must be F32 or BF16");
+  if (cache->dtype == LL_FP8_E4M3 ? in_dtype != LL_BF16 : in_dtype != cache->dtype)
+    return fail(LL_ERR_INVALID_ARG, "input dtype does not match the cache dtype");
+  if ((st = check_grid(rope, cache->tokens_per_frame)) != LL_OK) return st;
+  ll::AppendParams p{};
+  if ((st = make_rope(rope, cache->H, cache->D, first_frame, &p.rp)) != LL_OK) return st;
+  p.k_in = k;
+  p.v_in = v;
+  p.k_cache = cache->k;
+  p.v_cache = cache->v;
+  p.k_scale = cache->k_scale;
+  p.v_scale = cache->v_scale;
+  p.B = cache->B;
+  p.F = n_frames;
+  p.N = cache->tokens_per_frame;
+  p.H = cache->H;
+  p.D = cache->D;
+  p.n_sink = cache->n_sink;
+  p.n_local = cache->n_local;
+  p.first_frame = first_frame;
+  if (slots_out)
+    for (int i = 0; i < n_frames; ++i) ll_slot_of_frame(first_frame + i, cache->n_sink, cache->n_local, &slots_out[i]);
+  const long long chunks = static_cast<long long>(p.B) * n_frames * p.N * p.H * (p.D / 8);
+  const long long want = (chunks + 255) / 256;
+  const int grid = static_cast<int>(want < 8LL * num_sms() ? want : 8LL * num_sms());
+  const size_t smem = static_cast<size_t>(p.H) * (p.D / 2) * sizeof(float);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cache->dtype == LL_BF16)
+    ll::append_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 256, smem, s>>>(p);
+  else if (cache->dtype == LL_F32)
+    ll::append_kernel<float, float><<<grid, 256, smem, s>>>(p);
+  else
+    ll::append_kernel<__nv_bfloat16, uint8_t><<<grid, 256, smem, s>>>(p);
+  return check_launch("append_kernel");
+}
+
+size_t ll_sink_window_attention_workspace_bytes(const ll_kvcache* cache, int n_query_frames) {
+  (void)cache;
+  (void)n_query_frames;
+  return 0;
+}
+
+ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvcache* cache, long long first_frame,
+                                   int n_query_frames, const ll_rope_desc* rope, float softmax_scale, void* out,
+                                   float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  g_last_error.clear();
+  ll_status st = check_cache(cache);
+  if (st != LL_OK) return st;
+  if (q == nullptr || out == nullptr) return fail(LL_ERR_INVALID_ARG, "q and out must be non-NULL");
+  if (!aligned16(q) || !aligned16(out)) return fail(LL_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
+  if (first_frame < 0) return fail(LL_ERR_INVALID_ARG, "first_frame must be >= 0");
+  if (n_query_frames < 1 || n_query_frames > cache->n_local)
+    return fail(LL_ERR_INVALID_ARG, "n_query_frames = %d must lie in [1, n_local = %d]", n_query_frames,
+                cache->n_local);
+  if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale))
+    return fail(LL_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  const size_t need = ll_sink_window_attention_workspace_bytes(cache, n_query_frames);
+  if (workspace_bytes < need || (need > 0 && workspace == nullptr))
+    return fail(LL_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu required", workspace_bytes, need);
+  if ((st = check_grid(rope, cache->tokens_per_frame)) != LL_OK) return st;
+  const bool f32 = cache->dtype == LL_F32;
+  if (f32 ? q_dtype != LL_F32 : q_dtype != LL_BF16)
+    return fail(LL_ERR_INVALID_ARG, "q dtype must be F32 for an F32 cache and BF16 otherwise");
+  if (cache->dtype == LL_FP8_E4M3) return fail(LL_ERR_UNSUPPORTED, "attention over an FP8 cache is not built yet");
+  const long long S = cache->n_sink + cache->n_local;
+  const long long last = first_frame + n_query_frames - 1;
+  const long long valid_slots = last + 1 < S ? last + 1 : S;
+  ll::AttnParams p{};
+  if ((st = make_rope(rope, cache->H, cache->D, first_frame, &p.rp)) != LL_OK) return st;
+  p.q = q;
+  p.out = out;
+  p.lse = lse;
+  p.B = cache->B;
+  p.H = cache->H;
+  p.Tq = n_query_frames * cache->tokens_per_frame;
+  p.Nk = static_cast<int>(valid_slots * cache->tokens_per_frame);
+  p.softmax_scale = softmax_scale;
+  p.N = cache->tokens_per_frame;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!f32 && cache->D == 128) return launch_attention<ll::AttnTraits<128, __nv_bfloat16>>(p, cache, S, s);
+  if (!f32 && cache->D == 64) return launch_attention<ll::AttnTraits<64, __nv_bfloat16>>(p, cache, S, s);
+  if (f32 && cache->D == 64) return launch_attention<ll::AttnTraits<64, float>>(p, cache, S, s);
+  return fail(LL_ERR_UNSUPPORTED, "attention supports D = 64 or 128 (bf16) and D = 64 (f32); got D = %d", cache->D);
+}
+
+size_t ll_kv_recache_workspace_bytes(const ll_kvcache* cache, int d_model, int n_slots) {
+  (void)cache;
+  (void)d_model;
+  (void)n_slots;
+  return 0;
+}
+
+ll_status ll_kv_recache(const ll_kvcache* cache, const void* x, int d_model, const void* wk, const void* wv,
+                        const float* gamma, float rms_eps, const long long* slot_frames, int n_slots,
+                        const ll_rope_desc* rope, void* workspace, size_t workspace_bytes, void* stream) {
+  g_last_error.clear();
+  (void)cache; (void)x; (void)d_model; (void)wk; (void)wv; (void)gamma; (void)rms_eps;
+  (void)slot_frames; (void)n_slots; (void)rope; (void)workspace; (void)workspace_bytes; (void)stream;
+  return fail(LL_ERR_UNSUPPORTED, "kv recache is not built yet");
+}
+
+}  // extern "C"

@@ -1,0 +1,115 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/ll_api.h declares, maps frames to slots bit-exactly, and rejects bad
+arguments on the host before anything is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sink_window_attention_b200 as swa
+from oracle import window
+from tests.conftest import ROOT
+
+
+@pytest.fixture(scope="module")
+def L():
+    from sink_window_attention_b200 import build
+    build.build()
+    return swa.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "ll_api.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ll_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(swa.EXPORTED)
+    assert swa.abi_version() == 1
+
+
+@pytest.mark.parametrize("n_sink,n_local", [(3, 9), (0, 5), (2, 1), (4, 12)])
+def test_slot_map_bit_exact(L, n_sink, n_local):
+    for f in list(range(0, 300)) + [10**6 + 7, 2**40 + 3]:
+        assert swa.slot_of_frame(f, n_sink, n_local) == window.slot_of(f, n_sink, n_local)
+
+
+def test_slot_map_rejects(L):
+    with pytest.raises(swa.LLError) as e:
+        swa.slot_of_frame(-1)
+    assert e.value.status == swa.LL_ERR_INVALID_ARG
+
+
+def _cache(**kw):
+    c = swa.KVCacheC()
+    c.k, c.v = 4096, 8192            # fake device addresses: never dereferenced on these paths
+    c.k_scale = c.v_scale = None
+    c.dtype, c.B, c.H, c.D = swa.LL_BF16, 1, 12, 128
+    c.tokens_per_frame, c.n_sink, c.n_local = 1560, 3, 9
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def _rope(**kw):
+    r = swa.Rope(pairs=(22, 21, 21), grid_h=30, grid_w=52).to_c()
+    for k, v in kw.items():
+        setattr(r, k, v)
+    return r
+
+
+def _attn(L, cache, rope=None, first=0, nq=1, scale=0.0, ws=None, ws_bytes=0, q=1 << 20, out=1 << 21,
+          qdt=swa.LL_BF16):
+    return L.ll_sink_window_attention(q, qdt, ctypes.byref(cache), first, nq,
+                                      ctypes.byref(rope) if rope is not None else None, scale, out, None, ws,
+                                      ws_bytes, None)
+
+
+def test_attention_validation(L):
+    bad = [
+        dict(cache=_cache(k=None)),
+        dict(cache=_cache(D=100)),
+        dict(cache=_cache(H=65)),
+        dict(cache=_cache(n_local=0)),
+        dict(cache=_cache(dtype=swa.LL_FP8_E4M3)),            # FP8 without scales
+        dict(cache=_cache(), first=-1),
+        dict(cache=_cache(), nq=0),
+        dict(cache=_cache(), nq=10),
+        dict(cache=_cache(), scale=-1.0),
+        dict(cache=_cache(), q=None),
+        dict(cache=_cache(), q=(1 << 20) + 2),                 # misaligned
+        dict(cache=_cache(), qdt=swa.LL_F32),
+        dict(cache=_cache(), rope=_rope(pairs_t=10)),          # pairs do not sum to D/2
+        dict(cache=_cache(), rope=_rope(grid_w=51)),           # grid does not match N
+        dict(cache=_cache(), rope=_rope(theta0=0.5)),
+        dict(cache=_cache(), rope=_rope(sigma_t=1.5)),
+    ]
+    for kw in bad:
+        st = _attn(L, **kw)
+        assert st == swa.LL_ERR_INVALID_ARG, (kw, st)
+        assert swa.last_error() != ""
+
+
+def test_append_and_rope_validation(L):
+    k = v = 1 << 20
+    rc = ctypes.byref(_rope())
+    c = _cache()
+    slots = (ctypes.c_int * 16)()
+    assert L.ll_kvcache_append(ctypes.byref(c), None, v, swa.LL_BF16, 0, 1, rc, slots, None) == swa.LL_ERR_INVALID_ARG
+    assert L.ll_kvcache_append(ctypes.byref(c), k, v, swa.LL_BF16, 0, 10, rc, slots, None) == swa.LL_ERR_INVALID_ARG
+    assert L.ll_kvcache_append(ctypes.byref(c), k, v, swa.LL_F32, 0, 1, rc, slots, None) == swa.LL_ERR_INVALID_ARG
+    assert L.ll_kvcache_append(ctypes.byref(c), k, v, swa.LL_BF16, -3, 1, rc, slots, None) == swa.LL_ERR_INVALID_ARG
+    eps = (ctypes.c_float * 12)(*([0.0] * 11 + [1.5]))
+    r = _rope(sigma_t=0.8)
+    r.eps_h = ctypes.cast(eps, ctypes.POINTER(ctypes.c_float))
+    assert L.ll_kvcache_append(ctypes.byref(c), k, v, swa.LL_BF16, 0, 1, ctypes.byref(r), slots, None) == swa.LL_ERR_INVALID_ARG
+    assert "eps_h[11]" in swa.last_error()
+    assert L.ll_rope_apply(None, swa.LL_BF16, 1, 1, 12, 128, 0, rc, None) == swa.LL_ERR_INVALID_ARG
+    assert L.ll_rope_apply(k, swa.LL_FP8_E4M3, 1, 1, 12, 128, 0, rc, None) == swa.LL_ERR_INVALID_ARG
+    assert L.ll_rope_apply(k, swa.LL_BF16, 1, 1, 12, 128, 0, None, None) == swa.LL_ERR_INVALID_ARG
