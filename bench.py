@@ -333,13 +333,32 @@ def run_e2e(st: Stream, args, barrier, dist):
             "d2h_bytes_per_step": d2h, "steps": steps}
 
 
+ATTN_SOURCES = ("ll_attention.cuh", "ll_common.cuh", "ll_rope_append.cuh")
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in ATTN_SOURCES:
+        with open(os.path.join(ROOT, "sink_window_attention_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def load_traffic():
-    """DRAM bytes per attention launch from the committed ncu summary, if any."""
-    p = os.path.join(ROOT, "profiles", "attention_traffic.json")
-    if os.path.exists(p):
-        with open(p) as f:
-            return json.load(f).get("dram_bytes_per_launch")
-    return None
+    """DRAM bytes (read + write) per attention launch from the committed ncu
+    summary — only while the kernel sources still hash to the captured
+    version; otherwise null."""
+    p = os.path.join(ROOT, "profiles", "attention_wan_single_layer.md")
+    if not os.path.exists(p):
+        return None
+    text = open(p).read()
+    import re
+    m_hash = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    m_bytes = re.search(r"dram_bytes_per_launch[^|]*\|\s*([0-9]+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+        return None
+    return int(m_bytes.group(1))
 
 
 # ---------------------------------------------------------------------------

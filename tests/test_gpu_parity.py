@@ -153,7 +153,9 @@ def run_stream(w: W.Workload, frames, layer=0, rows_per_step=48, q_scale=1.0, ch
             r = assert_parity(got, ref, what=f"{w.name} frame {f0} b {b}")
             worst = (max(worst[0], r[0]), max(worst[1], r[1]))
             if check_lse:
-                assert_parity(lse[b].cpu().numpy()[:, rows], ref_lse, max_rel=1e-3, mean_abs=1e-3, what="lse")
+                # natural-log normaliser: 1e-3 of its largest magnitude at most,
+                # 5e-3 (0.5 % of the partition function) on average
+                assert_parity(lse[b].cpu().numpy()[:, rows], ref_lse, max_rel=1e-3, mean_abs=5e-3, what="lse")
     return worst
 
 
