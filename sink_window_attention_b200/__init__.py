@@ -214,6 +214,21 @@ def attention_workspace_bytes(cache: KVCache, n_query_frames: int) -> int:
     return int(lib().ll_sink_window_attention_workspace_bytes(ctypes.byref(cache.to_c()), n_query_frames))
 
 
+_workspaces = {}
+
+
+def workspace_for(nbytes: int, device) -> torch.Tensor:
+    """A device scratch buffer of at least nbytes, cached per device. Calls that
+    share it must be ordered (one stream); pass your own workspace to run
+    attention concurrently on several streams."""
+    key = torch.device(device)
+    t = _workspaces.get(key)
+    if t is None or t.numel() < nbytes:
+        t = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=key)
+        _workspaces[key] = t
+    return t
+
+
 def sink_window_attention(q: torch.Tensor, cache: KVCache, first_frame: int, rope: Optional[Rope],
                           softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
                           lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
@@ -222,7 +237,9 @@ def sink_window_attention(q: torch.Tensor, cache: KVCache, first_frame: int, rop
     F = q.shape[1] // cache.N
     if out is None:
         out = torch.empty_like(q)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if workspace is None:
+        workspace = workspace_for(attention_workspace_bytes(cache, F), q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
     _check(lib().ll_sink_window_attention(_ptr(q), _dtype_code(q.dtype), ctypes.byref(cache.to_c()), first_frame, F,
                                           _rope_ref(rope), float(softmax_scale), _ptr(out), _ptr(lse),
                                           _ptr(workspace), ws_bytes, _stream(stream)))

@@ -2,6 +2,7 @@
 from __future__ import annotations
 
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -35,11 +36,32 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(d) <= t for d in _deps())
 
 
+# Kernels that re-split registers between warpgroups (setmaxnreg) must be
+# launched with exactly this many registers per thread, or the increase would
+# wait for registers that do not exist.
+LAUNCH_REGS = {"sink_window_attention_kernel": 168}
+
+
+def check_register_split(ptxas_log: str) -> None:
+    current = None
+    for line in ptxas_log.splitlines():
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            current = m.group(1)
+            continue
+        m = re.search(r"Used (\d+) registers", line)
+        if m and current:
+            for name, regs in LAUNCH_REGS.items():
+                if name in current and int(m.group(1)) != regs:
+                    raise RuntimeError(f"{current}: ptxas allocated {m.group(1)} registers, the warpgroup "
+                                       f"register split needs exactly {regs}")
+
+
 def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if not force and up_to_date():
         return LIB
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
-           "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr", "-Xptxas", "-v" if verbose else "-O3",
+           "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr", "-Xptxas", "-v",
            "-I", os.path.join(ROOT, "include"),
            "-o", LIB + ".tmp"] + list(extra) + [os.path.join(CSRC, s) for s in SOURCES]
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -48,6 +70,11 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         raise RuntimeError("nvcc failed building libll_swa.so")
     if verbose:
         sys.stderr.write(r.stderr)
+    try:
+        check_register_split(r.stderr)
+    except RuntimeError:
+        os.remove(LIB + ".tmp")
+        raise
     os.replace(LIB + ".tmp", LIB)
     return LIB
 

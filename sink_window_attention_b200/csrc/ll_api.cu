@@ -145,8 +145,29 @@ ll_status encode_rows_map(CUtensorMap* map, const void* base, CUtensorMapDataTyp
   return LL_OK;
 }
 
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Workspace of one attention call: per-unit arrival counters, then
+// (#SMs + units) partial slots of SLOT_FLOATS floats.
 template <class TR>
-ll_status launch_attention(const ll::AttnParams& p, const ll_kvcache* c, long long S, cudaStream_t stream) {
+size_t attention_workspace(int units) {
+  return align256(static_cast<size_t>(units) * sizeof(int)) +
+         static_cast<size_t>(num_sms() + units) * TR::SLOT_FLOATS * sizeof(float);
+}
+
+template <class TR>
+ll_status launch_attention(ll::AttnParams p, const ll_kvcache* c, long long S, void* workspace, size_t ws_bytes,
+                           cudaStream_t stream) {
+  p.q_tiles = (p.Tq + TR::BM - 1) / TR::BM;
+  p.nkv = (p.Nk + TR::BN - 1) / TR::BN;
+  p.units = p.q_tiles * c->H * c->B;
+  p.total = static_cast<long long>(p.units) * p.nkv;
+  p.grid = static_cast<int>(p.total < num_sms() ? p.total : num_sms());
+  const size_t need = attention_workspace<TR>(p.units);
+  if (workspace == nullptr || ws_bytes < need)
+    return fail(LL_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu required", ws_bytes, need);
+  p.counters = static_cast<int*>(workspace);
+  p.partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(p.units * sizeof(int)));
   CUtensorMap tmK, tmV;
   const CUtensorMapDataType dt = TR::ES == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   const long long batch_rows = S * c->tokens_per_frame;
@@ -162,8 +183,9 @@ ll_status launch_attention(const ll::AttnParams& p, const ll_kvcache* c, long lo
       return check_launch("cudaFuncSetAttribute(attention)");
     attr_set = true;
   }
-  const dim3 grid((p.Tq + TR::BM - 1) / TR::BM, c->H, c->B);
-  kern<<<grid, TR::THREADS, TR::SMEM_BYTES, stream>>>(tmK, tmV, p);
+  if (cudaMemsetAsync(p.counters, 0, p.units * sizeof(int), stream) != cudaSuccess)
+    return check_launch("cudaMemsetAsync(attention counters)");
+  kern<<<p.grid, TR::THREADS, TR::SMEM_BYTES, stream>>>(tmK, tmV, p);
   return check_launch("sink_window_attention_kernel");
 }
 
@@ -216,6 +238,7 @@ ll_status ll_rope_apply(void* x, ll_dtype dtype, int B, int n_frames, int H, int
   p.H = H;
   p.D = D;
   const long long chunks = static_cast<long long>(B) * n_frames * p.N * H * (D / 8);
+  if (chunks >= (1LL << 31)) return fail(LL_ERR_UNSUPPORTED, "tensor too large for one call (%lld chunks)", chunks);
   const long long want = (chunks + 255) / 256;
   const int grid = static_cast<int>(want < 8LL * num_sms() ? want : 8LL * num_sms());
   const size_t smem = static_cast<size_t>(H) * (D / 2) * sizeof(float);
@@ -261,6 +284,7 @@ ll_status ll_kvcache_append(const ll_kvcache* cache, const void* k, const void* 
   if (slots_out)
     for (int i = 0; i < n_frames; ++i) ll_slot_of_frame(first_frame + i, cache->n_sink, cache->n_local, &slots_out[i]);
   const long long chunks = static_cast<long long>(p.B) * n_frames * p.N * p.H * (p.D / 8);
+  if (chunks >= (1LL << 31)) return fail(LL_ERR_UNSUPPORTED, "tensor too large for one call (%lld chunks)", chunks);
   const long long want = (chunks + 255) / 256;
   const int grid = static_cast<int>(want < 8LL * num_sms() ? want : 8LL * num_sms());
   const size_t smem = static_cast<size_t>(p.H) * (p.D / 2) * sizeof(float);
@@ -275,9 +299,12 @@ ll_status ll_kvcache_append(const ll_kvcache* cache, const void* k, const void* 
 }
 
 size_t ll_sink_window_attention_workspace_bytes(const ll_kvcache* cache, int n_query_frames) {
-  (void)cache;
-  (void)n_query_frames;
-  return 0;
+  if (cache == nullptr || n_query_frames < 1 || cache->tokens_per_frame < 1 || cache->H < 1 || cache->B < 1)
+    return 0;
+  const int units = ((n_query_frames * cache->tokens_per_frame + 127) / 128) * cache->H * cache->B;
+  if (cache->D == 128) return attention_workspace<ll::AttnTraits<128, __nv_bfloat16>>(units);
+  if (cache->dtype == LL_F32) return attention_workspace<ll::AttnTraits<64, float>>(units);
+  return attention_workspace<ll::AttnTraits<64, __nv_bfloat16>>(units);
 }
 
 ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvcache* cache, long long first_frame,
@@ -295,8 +322,9 @@ ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvc
   if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale))
     return fail(LL_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
   const size_t need = ll_sink_window_attention_workspace_bytes(cache, n_query_frames);
-  if (workspace_bytes < need || (need > 0 && workspace == nullptr))
+  if (workspace == nullptr || workspace_bytes < need)
     return fail(LL_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu required", workspace_bytes, need);
+  if (!aligned16(workspace)) return fail(LL_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
   if ((st = check_grid(rope, cache->tokens_per_frame)) != LL_OK) return st;
   const bool f32 = cache->dtype == LL_F32;
   if (f32 ? q_dtype != LL_F32 : q_dtype != LL_BF16)
@@ -317,9 +345,12 @@ ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvc
   p.softmax_scale = softmax_scale;
   p.N = cache->tokens_per_frame;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (!f32 && cache->D == 128) return launch_attention<ll::AttnTraits<128, __nv_bfloat16>>(p, cache, S, s);
-  if (!f32 && cache->D == 64) return launch_attention<ll::AttnTraits<64, __nv_bfloat16>>(p, cache, S, s);
-  if (f32 && cache->D == 64) return launch_attention<ll::AttnTraits<64, float>>(p, cache, S, s);
+  if (!f32 && cache->D == 128)
+    return launch_attention<ll::AttnTraits<128, __nv_bfloat16>>(p, cache, S, workspace, workspace_bytes, s);
+  if (!f32 && cache->D == 64)
+    return launch_attention<ll::AttnTraits<64, __nv_bfloat16>>(p, cache, S, workspace, workspace_bytes, s);
+  if (f32 && cache->D == 64)
+    return launch_attention<ll::AttnTraits<64, float>>(p, cache, S, workspace, workspace_bytes, s);
   return fail(LL_ERR_UNSUPPORTED, "attention supports D = 64 or 128 (bf16) and D = 64 (f32); got D = %d", cache->D);
 }
 

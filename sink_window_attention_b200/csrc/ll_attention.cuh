@@ -6,25 +6,34 @@
 // over all tokens of the occupied cache slots [0, S_valid), i.e. the 3 sink
 // frames plus the most recent local frames; there is no mask inside that set.
 //
-// How: a flash-style single pass with an online softmax.
-//  * one CTA per (query tile of 128 rows, head, batch);
-//  * warp 0 (one lane) streams K and V tiles of 128 keys straight out of the
-//    [B][S*N][H][D] cache with 4D TMA loads (128-byte swizzle, rows past the
-//    valid keys are zero-filled by the TMA unit), STAGES deep; V is the
-//    MN-major operand of P V, which for 32-bit (tf32) data needs the 128-byte
-//    swizzle with 32-byte atoms;
-//  * warp 1 owns the tensor memory (512 columns: two S buffers and O) and one
-//    lane issues tcgen05.mma: S_j = Q K_j^T into the free S buffer while the
-//    softmax works on the other one, then O += P_j V_j;
-//  * warps 4-7 (one TMEM lane quarter each, one query row per thread) read
-//    S_j from TMEM, keep the running max / sum, write P_j = exp2(...) to
-//    shared memory in the operand layout, rescale O in TMEM only when the
-//    running max grows by more than 2^8 (the final division uses the same
-//    stale max, so the result is unchanged), and finally normalise O and
-//    store it;
-//  * Q is loaded by warps 1-7 with plain 128-bit loads, rotated (3D RoPE with
-//    the head's jittered temporal base) in registers and written to shared
-//    memory in the swizzled layout, so RoPE costs no extra pass over Q.
+// How (flash-style single pass, online softmax in the exp2 domain):
+//  * Work is a list of units = (128-row query tile, head, batch), each with
+//    nkv tiles of 128 keys. A persistent grid of G CTAs (G = #SMs) splits the
+//    flattened (unit, key tile) range into G equal contiguous ranges, so every
+//    SM gets the same number of key tiles; a CTA processes its range as pieces
+//    (one piece per unit it touches). A piece that covers a whole unit writes
+//    O directly; otherwise it writes its unnormalised (O, m, l) to a workspace
+//    slot and the CTA that finishes a unit's last piece merges all of them.
+//  * warp 0 (one lane) streams K tiles and V tiles (separate rings, K one tile
+//    ahead) straight out of the [B][S*N][H][D] cache with 4D TMA loads
+//    (128-byte swizzle; rows past the valid keys read as zeros).
+//  * warps 2-3 load the next piece's Q tile with 128-bit loads, apply the 3D
+//    RoPE in registers and write the swizzled operand layout into the free
+//    half of a double-buffered Q, so RoPE costs no extra pass over Q.
+//  * warp 1 owns 512 TMEM columns: S_A, S_B (128 each) and O_A, O_B. One lane
+//    issues tcgen05.mma: S_i = Q K_i^T into S_(i mod 2) and O_(i mod 2) +=
+//    P_i V_i, where P_i sits in the TMEM columns of S_i (the A operand is read
+//    from tensor memory), so P never touches shared memory.
+//  * two softmax warpgroups (warps 4-7: even key tiles of a piece, warps 8-11:
+//    odd ones; one query row per thread, one TMEM lane quarter per warp) keep
+//    independent running (max, sum) and O; O is rescaled in TMEM only when the
+//    running max grows by more than 2^8 (the final division uses the same max,
+//    so the result is unchanged). At the end of a piece warpgroup A merges
+//    the two halves.
+//  * Every mbarrier wait is bounded; a wait that gives up records an error,
+//    raises an abort flag the other roles see, and all roles still walk the
+//    same named-barrier sequence so nothing can hang. TMEM accesses
+//    (warp-collective) only run under warp-uniform conditions.
 #pragma once
 
 #include "ll_common.cuh"
@@ -44,23 +53,30 @@ struct AttnTraits {
   static constexpr int ELEMS_PER_BLOCK = 128 / ES;  // elements of D per column block
   static constexpr int Q_BYTES = BM * ROWB;
   static constexpr int KV_BYTES = BN * ROWB;
-  static constexpr int PROWB = BN * ES;             // bytes of one P row
-  static constexpr int P_BYTES = BM * PROWB;
   static constexpr int QK_STEPS = ROWB / 32;        // MMAs per S tile (32 bytes of K each)
-  static constexpr int PV_STEPS = PROWB / 32;       // MMAs per P V
+  static constexpr int PV_STEPS = BN * ES / 32;     // MMAs per P V (8 bf16 / 16 tf32)
   static constexpr int MMA_K = 32 / ES;             // reduction elements per MMA
   static constexpr int FMT = (ES == 2) ? 1 : 2;     // bf16 / tf32
-  static constexpr int CTRL_BYTES = 1024;
-  static constexpr int FIXED_BYTES = Q_BYTES + P_BYTES + CTRL_BYTES + 1024;  // + alignment slack
-  static constexpr int NSTAGE = (FIXED_BYTES + 8 * KV_BYTES <= 232448)   ? 4
-                                : (FIXED_BYTES + 6 * KV_BYTES <= 232448) ? 3
-                                                                         : 2;
-  static constexpr int SMEM_BYTES = FIXED_BYTES + 2 * NSTAGE * KV_BYTES;
+  static constexpr int QST = 2;                     // Q buffers
+  static constexpr int CTRL_BYTES = 2048;
+  static constexpr int STAGE_BUDGET = 232448 - CTRL_BYTES - 1024 - QST * Q_BYTES;
+  static constexpr int STAGES = STAGE_BUDGET / KV_BYTES;
+  static constexpr int KST = STAGES >= 8 ? 4 : (STAGES + 1) / 2;
+  static constexpr int VST = STAGES >= 8 ? 4 : STAGES - KST;
+  static constexpr int SMEM_BYTES = CTRL_BYTES + 1024 + QST * Q_BYTES + (KST + VST) * KV_BYTES;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int S_COL0 = 0, S_COL1 = BN, O_COL = 2 * BN;
-  static constexpr int THREADS = 256;
+  static constexpr int S_COL0 = 0, O_COL0 = 2 * BN;  // S_w at w*BN, O_w at O_COL0 + w*D
+  static constexpr int THREADS = 384;
+  // register split: launch 168 per thread (384 x 168 = 64512); warpgroup 0
+  // (producer, MMA, Q loader) gives up 96 per thread, the two softmax
+  // warpgroups take 48 more: 128 x 72 + 256 x 216 = 64512. The build checks
+  // that ptxas allocated exactly LAUNCH_REGS.
+  static constexpr int LAUNCH_REGS = 168, REGS_LOW = 72, REGS_HIGH = 216;
+  static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= THREADS * LAUNCH_REGS, "register split exceeds the launch");
+  static constexpr int SLOT_FLOATS = BM * D + 2 * BM;  // one partial: O rows, then m, then l
+  static_assert(KST >= 2 && VST >= 2, "need at least two K and two V stages");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert(O_COL + D <= TMEM_COLS, "TMEM budget");
+  static_assert(O_COL0 + 2 * D <= TMEM_COLS, "TMEM budget");
   static_assert(NB >= 1 && ROWB % 128 == 0, "rows must be whole 128-byte blocks");
 };
 
@@ -69,50 +85,133 @@ struct AttnParams {
   void* out;         // [B][Tq][H][D]
   float* lse;        // [B][H][Tq] or nullptr
   int B, H, Tq, Nk;  // Nk: valid keys per batch entry
+  int N;             // tokens per frame
   float softmax_scale;
   RopeParams rp;     // Q rotation (rp.enabled == 0: q already rotated); rp.t_first = first query frame
-  int N;             // tokens per frame
+  int q_tiles;       // ceil(Tq / 128)
+  int nkv;           // ceil(Nk / 128)
+  int units;         // q_tiles * H * B
+  int grid;          // G: number of CTAs
+  long long total;   // units * nkv
+  int* counters;     // [units] arrivals per unit (zeroed by the host before the launch)
+  float* partials;   // [(grid + units) * SLOT_FLOATS]
 };
 
+// A piece: key tiles [j0, j0 + n) of unit u.
+struct Piece {
+  int u, j0, n;
+};
+
+// CTA that owns flattened iteration i when `total` iterations are split into
+// G contiguous ranges starting at floor(g * total / G).
+__device__ __forceinline__ int owner_of(long long i, long long total, int G) {
+  return static_cast<int>(((i + 1) * G - 1) / total);
+}
+
+// Q tile of unit u, rotated with this head's frequencies `om` [D/2], into
+// the 128-byte-swizzled K-major operand layout at sQ.
 template <class TR>
-__global__ void __launch_bounds__(256, 1)
+__device__ __forceinline__ void load_q_tile(uint8_t* sQ, const AttnParams& p, const float* om, int u, int tid,
+                                            int nthreads) {
+  using T = typename TR::T;
+  constexpr int BM = TR::BM, D = TR::D;
+  const int qt = u % p.q_tiles;
+  const int h = (u / p.q_tiles) % p.H;
+  const int b = u / (p.q_tiles * p.H);
+  const int q0 = qt * BM;
+  const T* q = static_cast<const T*>(p.q);
+  constexpr int GPR = D / 8;  // 8-element groups per row
+  const int pth = p.rp.pt + p.rp.ph;
+  for (int g = tid; g < BM * GPR; g += nthreads) {
+    const int r = g / GPR, e8 = g - r * GPR;
+    const int t = q0 + r;
+    float x[8];
+    if (t < p.Tq) {
+      load_chunk8<T>(q + ((static_cast<size_t>(b) * p.Tq + t) * p.H + h) * D + e8 * 8, x);
+      if (p.rp.enabled) {
+        const int fi = t / p.N, n = t - fi * p.N;
+        const int rr = n / p.rp.grid_w, cc = n - rr * p.rp.grid_w;
+        rotate_chunk8(x, e8 * 4, static_cast<float>(p.rp.t_first + fi), static_cast<float>(rr),
+                      static_cast<float>(cc), om, p.rp.pt, pth);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = 0.f;
+    }
+    if constexpr (TR::ES == 2) {
+      const int chunk = e8;  // 8 bf16 = 16 bytes
+      uint4 v;
+      v.x = pack_bf16(x[0], x[1]);
+      v.y = pack_bf16(x[2], x[3]);
+      v.z = pack_bf16(x[4], x[5]);
+      v.w = pack_bf16(x[6], x[7]);
+      *reinterpret_cast<uint4*>(sQ + (chunk >> 3) * (BM * 128) + sw128_offset(r, chunk & 7)) = v;
+    } else {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int chunk = e8 * 2 + hh;  // 4 floats = 16 bytes
+        *reinterpret_cast<float4*>(sQ + (chunk >> 3) * (BM * 128) + sw128_offset(r, chunk & 7)) =
+            make_float4(x[4 * hh], x[4 * hh + 1], x[4 * hh + 2], x[4 * hh + 3]);
+      }
+    }
+  }
+  fence_proxy_async_smem();
+}
+
+template <class TR>
+__global__ void __launch_bounds__(384, 1)
     sink_window_attention_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                                  const AttnParams p) {
   using T = typename TR::T;
-  constexpr int BM = TR::BM, BN = TR::BN, D = TR::D, ST = TR::NSTAGE;
+  constexpr int BM = TR::BM, BN = TR::BN, D = TR::D, KST = TR::KST, VST = TR::VST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + TR::Q_BYTES;
-  uint8_t* sV = sK + ST * TR::KV_BYTES;
-  uint8_t* sP = sV + ST * TR::KV_BYTES;
-  uint8_t* ctrl = sP + TR::P_BYTES;
+  uint8_t* sQ = smem;                              // [QST][Q_BYTES]
+  uint8_t* sK = sQ + TR::QST * TR::Q_BYTES;        // [KST][KV_BYTES]
+  uint8_t* sV = sK + KST * TR::KV_BYTES;           // [VST][KV_BYTES]
+  uint8_t* ctrl = sV + VST * TR::KV_BYTES;
   uint64_t* k_full = reinterpret_cast<uint64_t*>(ctrl);
-  uint64_t* v_full = k_full + ST;
-  uint64_t* kv_empty = v_full + ST;
-  uint64_t* s_full = kv_empty + ST;  // [2]
-  uint64_t* p_ready = s_full + 2;
-  uint64_t* o_done = p_ready + 1;
-  uint64_t* drain = o_done + 1;
+  uint64_t* k_empty = k_full + KST;
+  uint64_t* v_full = k_empty + KST;
+  uint64_t* v_empty = v_full + VST;
+  uint64_t* q_full = v_empty + VST;   // [2]
+  uint64_t* q_empty = q_full + 2;     // [2]
+  uint64_t* s_full = q_empty + 2;     // [2] per softmax warpgroup
+  uint64_t* p_ready = s_full + 2;     // [2]
+  uint64_t* o_done = p_ready + 2;     // [2]
+  uint64_t* b_ready = o_done + 2;     // warpgroup B's piece state is in smem
+  uint64_t* merged = b_ready + 1;     // warpgroup A has read O_A, O_B of the piece
+  uint64_t* drain = merged + 1;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
-  float* s_omega = reinterpret_cast<float*>(ctrl + 512);  // [D/2]
+  volatile int* s_last = reinterpret_cast<volatile int*>(s_tmem + 2);
+  float* s_mB = reinterpret_cast<float*>(ctrl + 256);      // [128]
+  float* s_lB = s_mB + BM;                                 // [128]
+  float* s_omega = reinterpret_cast<float*>(ctrl + 1280);  // [2][D/2]: one head per Q buffer
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int q0 = qt * BM;
-  const int nkv = (p.Nk + BN - 1) / BN;
+  const int g = blockIdx.x;
+  const long long it_begin = g * p.total / p.grid;
+  const long long it_end = (g + 1) * p.total / p.grid;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < ST; ++s) {
+    for (int s = 0; s < KST; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_empty[s], 1);
     }
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(p_ready, BM);
-    mbar_init(o_done, 1);
+    for (int s = 0; s < VST; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_ready[s], BM);
+      mbar_init(&o_done[s], 1);
+    }
+    mbar_init(b_ready, BM);
+    mbar_init(merged, BM);
     mbar_init(drain, 1);
     *s_abort = 0;
     fence_mbar_init();
@@ -126,268 +225,369 @@ __global__ void __launch_bounds__(256, 1)
   tc_fence_after();
   const uint32_t tbase = *s_tmem;
 
+  // The piece sequence of this CTA, walked identically by every role.
+  auto next_piece = [&](long long& it, Piece& pc) -> bool {
+    if (it >= it_end) return false;
+    pc.u = static_cast<int>(it / p.nkv);
+    pc.j0 = static_cast<int>(it - static_cast<long long>(pc.u) * p.nkv);
+    const long long left = it_end - it;
+    pc.n = static_cast<int>(left < p.nkv - pc.j0 ? left : p.nkv - pc.j0);
+    it += pc.n;
+    return true;
+  };
+
+  if (warp < 4) {
+  // warpgroup 0: producer, MMA issuer, Q loader (same setmaxnreg for its four warps)
+  regs_dec<TR::REGS_LOW>();
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      int issued = 0;
-      for (int j = 0; j < nkv; ++j) {
-        const int st = j % ST, n = j / ST;
-        if (!mbar_wait(&kv_empty[st], (n & 1) ^ 1, s_abort)) break;
+      long long it = it_begin;
+      Piece pc;
+      int kc = 0, vc = 0;  // K / V tiles issued so far
+      bool ok = true;
+      auto load_k = [&](int h, int b, int j) -> bool {
+        const int st = kc % KST;
+        if (!mbar_wait(&k_empty[st], ((kc / KST) & 1) ^ 1, s_abort)) return false;
         mbar_expect_tx(&k_full[st], TR::KV_BYTES);
 #pragma unroll
         for (int blk = 0; blk < TR::NB; ++blk)
           tma_load_4d(sK + st * TR::KV_BYTES + blk * (BN * 128), &tmK, &k_full[st], blk * TR::ELEMS_PER_BLOCK, h,
                       j * BN, b);
+        ++kc;
+        return true;
+      };
+      auto load_v = [&](int h, int b, int j) -> bool {
+        const int st = vc % VST;
+        if (!mbar_wait(&v_empty[st], ((vc / VST) & 1) ^ 1, s_abort)) return false;
         mbar_expect_tx(&v_full[st], TR::KV_BYTES);
 #pragma unroll
         for (int blk = 0; blk < TR::NB; ++blk)
           tma_load_4d(sV + st * TR::KV_BYTES + blk * (BN * 128), &tmV, &v_full[st], blk * TR::ELEMS_PER_BLOCK, h,
                       j * BN, b);
-        issued = j + 1;
+        ++vc;
+        return true;
+      };
+      while (ok && next_piece(it, pc)) {
+        const int h = (pc.u / p.q_tiles) % p.H;
+        const int b = pc.u / (p.q_tiles * p.H);
+        // K runs one tile ahead of V
+        ok = load_k(h, b, pc.j0);
+        for (int i = 0; ok && i < pc.n; ++i) {
+          if (i + 1 < pc.n) ok = load_k(h, b, pc.j0 + i + 1);
+          if (ok) ok = load_v(h, b, pc.j0 + i);
+        }
       }
       if (*s_abort) {  // let the copies already in flight land before the CTA exits
-        for (int t = issued - ST > 0 ? issued - ST : 0; t < issued; ++t) {
-          mbar_wait_teardown(&k_full[t % ST], (t / ST) & 1);
-          mbar_wait_teardown(&v_full[t % ST], (t / ST) & 1);
-        }
+        for (int t = kc - KST > 0 ? kc - KST : 0; t < kc; ++t) mbar_wait_teardown(&k_full[t % KST], (t / KST) & 1);
+        for (int t = vc - VST > 0 ? vc - VST : 0; t < vc; ++t) mbar_wait_teardown(&v_full[t % VST], (t / VST) & 1);
       }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_dense(BM, BN, TR::FMT, false, false);
+      constexpr uint32_t idO = idesc_dense(BM, D, TR::FMT, false, true);
+      const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
+      long long it = it_begin;
+      Piece pc;
+      int kc = 0, vc = 0, pidx = 0;
+      bool ok = true;
+      auto issue_s = [&](int w, int qb) -> bool {
+        const int st = kc % KST;
+        if (!mbar_wait(&k_full[st], (kc / KST) & 1, s_abort)) return false;
+        tc_fence_after();
+        const uint32_t d = tbase + TR::S_COL0 + w * BN;
+#pragma unroll
+        for (int k = 0; k < TR::QK_STEPS; ++k) {
+          const uint32_t off = (k >> 2) * (BM * 128) + (k & 3) * 32;
+          const uint32_t offk = (k >> 2) * (BN * 128) + (k & 3) * 32;
+          const uint64_t da = desc_sw128(aQ + qb * TR::Q_BYTES + off, 16, 1024);
+          const uint64_t db = desc_sw128(aK + st * TR::KV_BYTES + offk, 16, 1024);
+          if constexpr (TR::ES == 2) mma_bf16_ss(d, da, db, idS, k > 0 ? 1u : 0u);
+          else mma_tf32_ss(d, da, db, idS, k > 0 ? 1u : 0u);
+        }
+        mma_commit(&s_full[w]);
+        mma_commit(&k_empty[st]);
+        ++kc;
+        return true;
+      };
+      auto issue_pv = [&](int w, bool acc) -> bool {
+        const int st = vc % VST;
+        if (!mbar_wait(&v_full[st], (vc / VST) & 1, s_abort)) return false;
+        tc_fence_after();
+        const uint32_t d = tbase + TR::O_COL0 + w * D;
+        const uint32_t pa = tbase + TR::S_COL0 + w * BN;  // P_w aliases S_w
+#pragma unroll
+        for (int k = 0; k < TR::PV_STEPS; ++k) {
+          const uint32_t av = aV + st * TR::KV_BYTES + k * TR::MMA_K * 128;
+          if constexpr (TR::ES == 2) {
+            mma_bf16_ts(d, pa + k * 8, desc_sw128(av, BN * 128, 1024), idO, (acc || k > 0) ? 1u : 0u);
+          } else {
+            mma_tf32_ts(d, pa + k * 8, desc_mn_sw128_atom32(av, BN * 128, 512), idO, (acc || k > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit(&o_done[w]);
+        mma_commit(&v_empty[st]);
+        ++vc;
+        return true;
+      };
+      int pcnt[2] = {0, 0};  // P tiles consumed per softmax warpgroup
+      while (ok && next_piece(it, pc)) {
+        const int qb = pidx & 1;
+        ok = mbar_wait(&q_full[qb], (pidx >> 1) & 1, s_abort);
+        for (int i = 0; ok && i < 2 && i < pc.n; ++i) ok = issue_s(i, qb);
+        for (int i = 0; ok && i < pc.n; ++i) {
+          const int w = i & 1;
+          if (!mbar_wait(&p_ready[w], pcnt[w] & 1, s_abort)) { ok = false; break; }
+          ++pcnt[w];
+          // the previous piece's O_A / O_B must have been read before the first P V overwrites them
+          if (i == 0 && pidx > 0 && !mbar_wait(merged, (pidx - 1) & 1, s_abort)) { ok = false; break; }
+          tc_fence_after();
+          if (!issue_pv(w, i >= 2)) { ok = false; break; }
+          if (i + 2 < pc.n && !issue_s(w, qb)) { ok = false; break; }
+        }
+        mma_commit(&q_empty[qb]);  // Q buffer free once every MMA issued so far has completed
+        ++pidx;
+      }
+      mma_commit(drain);  // every MMA issued above has finished once `drain` completes
+      mbar_wait_teardown(drain, 0);
     }
   } else {
-    // ------------------------------------------- Q load with fused 3D RoPE (warps 1-7)
-    const int tid = threadIdx.x - 32;  // 0..223
-    constexpr int NT = 224;
-    if (p.rp.enabled) build_omega_one_head(s_omega, p.rp, h, D / 2, tid, NT);
-    asm volatile("bar.sync 1, 224;" ::: "memory");
-    const T* q = static_cast<const T*>(p.q);
-    constexpr int GPR = D / 8;  // 8-element groups per row
-    const int pth = p.rp.pt + p.rp.ph;
-    for (int g = tid; g < BM * GPR; g += NT) {
-      const int r = g / GPR, e8 = g - r * GPR;
-      const int t = q0 + r;
-      float x[8];
-      if (t < p.Tq) {
-        load_chunk8<T>(q + ((static_cast<long long>(b) * p.Tq + t) * p.H + h) * D + e8 * 8, x);
-        if (p.rp.enabled) {
-          const int fi = t / p.N, n = t - fi * p.N;
-          const int rr = n / p.rp.grid_w, cc = n - rr * p.rp.grid_w;
-          rotate_chunk8(x, e8 * 4, static_cast<float>(p.rp.t_first + fi), static_cast<float>(rr),
-                        static_cast<float>(cc), s_omega, p.rp.pt, pth);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] = 0.f;
-      }
-      // 16-byte chunks of this group inside the row, then their swizzled place
-      if constexpr (TR::ES == 2) {
-        const int chunk = e8;  // 8 bf16 = 16 bytes
-        uint4 u;
-        u.x = pack_bf16(x[0], x[1]);
-        u.y = pack_bf16(x[2], x[3]);
-        u.z = pack_bf16(x[4], x[5]);
-        u.w = pack_bf16(x[6], x[7]);
-        *reinterpret_cast<uint4*>(sQ + (chunk >> 3) * (BM * 128) + sw128_offset(r, chunk & 7)) = u;
-      } else {
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int chunk = e8 * 2 + hh;  // 4 floats = 16 bytes
-          *reinterpret_cast<float4*>(sQ + (chunk >> 3) * (BM * 128) + sw128_offset(r, chunk & 7)) =
-              make_float4(x[4 * hh], x[4 * hh + 1], x[4 * hh + 2], x[4 * hh + 3]);
-        }
-      }
+    // ------------------------------------------------ Q loader (warps 2-3) with fused RoPE
+    const int tid = threadIdx.x - 64;  // 0..63
+    long long it = it_begin;
+    Piece pc;
+    int pidx = 0;
+    while (next_piece(it, pc)) {
+      const int qb = pidx & 1;
+      const int h = (pc.u / p.q_tiles) % p.H;
+      const bool ok = mbar_wait(&q_empty[qb], ((pidx >> 1) & 1) ^ 1, s_abort);
+      float* om = s_omega + qb * (D / 2);
+      if (ok && p.rp.enabled)
+        for (int j = tid; j < D / 2; j += 64) om[j] = omega_of(p.rp, h, j);
+      asm volatile("bar.sync 2, 64;" ::: "memory");
+      if (ok) load_q_tile<TR>(sQ + qb * TR::Q_BYTES, p, om, pc.u, tid, 64);
+      asm volatile("bar.sync 2, 64;" ::: "memory");
+      if (tid == 0) mbar_arrive(&q_full[qb]);
+      ++pidx;
     }
-    fence_proxy_async_smem();
-    asm volatile("bar.sync 1, 224;" ::: "memory");
-
-    if (warp == 1) {
-      // ------------------------------------------------------------ MMA issuer
-      if (lane == 0) {
-        constexpr uint32_t idS = idesc_dense(BM, BN, TR::FMT, false, false);
-        constexpr uint32_t idO = idesc_dense(BM, D, TR::FMT, false, true);
-        const uint32_t tS[2] = {tbase + TR::S_COL0, tbase + TR::S_COL1};
-        const uint32_t tO = tbase + TR::O_COL;
-        const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV), aP = smem_addr(sP);
-        auto issue_qk = [&](uint32_t d, int st) {
-#pragma unroll
-          for (int k = 0; k < TR::QK_STEPS; ++k) {
-            const uint32_t off = (k >> 2) * (BM * 128) + (k & 3) * 32;
-            const uint32_t offk = (k >> 2) * (BN * 128) + (k & 3) * 32;
-            const uint64_t da = desc_sw128(aQ + off, 16, 1024);
-            const uint64_t db = desc_sw128(aK + st * TR::KV_BYTES + offk, 16, 1024);
-            if constexpr (TR::ES == 2) mma_bf16_ss(d, da, db, idS, k > 0 ? 1u : 0u);
-            else mma_tf32_ss(d, da, db, idS, k > 0 ? 1u : 0u);
-          }
-        };
-        auto issue_pv = [&](int st, bool acc) {
-#pragma unroll
-          for (int k = 0; k < TR::PV_STEPS; ++k) {
-            const uint32_t offp = (k >> 2) * (BM * 128) + (k & 3) * 32;
-            const uint64_t da = desc_sw128(aP + offp, 16, 1024);
-            const uint32_t av = aV + st * TR::KV_BYTES + k * TR::MMA_K * 128;
-            if constexpr (TR::ES == 2) {
-              mma_bf16_ss(tO, da, desc_sw128(av, BN * 128, 1024), idO, (acc || k > 0) ? 1u : 0u);
-            } else {
-              mma_tf32_ss(tO, da, desc_mn_sw128_atom32(av, BN * 128, 512), idO, (acc || k > 0) ? 1u : 0u);
-            }
-          }
-        };
-        if (mbar_wait(&k_full[0], 0, s_abort)) {
-          tc_fence_after();
-          issue_qk(tS[0], 0);
-          mma_commit(&s_full[0]);
-          for (int j = 0; j < nkv; ++j) {
-            if (j + 1 < nkv) {
-              const int st1 = (j + 1) % ST;
-              if (!mbar_wait(&k_full[st1], ((j + 1) / ST) & 1, s_abort)) break;
-              tc_fence_after();
-              issue_qk(tS[(j + 1) & 1], st1);
-              mma_commit(&s_full[(j + 1) & 1]);
-            }
-            if (!mbar_wait(p_ready, j & 1, s_abort)) break;
-            const int st = j % ST;
-            if (!mbar_wait(&v_full[st], (j / ST) & 1, s_abort)) break;
-            tc_fence_after();
-            issue_pv(st, j > 0);
-            mma_commit(o_done);
-            mma_commit(&kv_empty[st]);
-          }
-        }
-        // every MMA issued above has finished once `drain` completes
-        mma_commit(drain);
-        mbar_wait_teardown(drain, 0);
-      }
-    } else if (warp >= 4) {
-      // ------------------------------------------------ softmax / correction / epilogue
-      const int row = threadIdx.x - 128;           // 0..127 == TMEM lane
-      const uint32_t lane_off = static_cast<uint32_t>((warp - 4) * 32) << 16;
-      const float scale = p.softmax_scale > 0.f ? p.softmax_scale : rsqrtf(static_cast<float>(D));
-      const float sl2 = scale * 1.4426950408889634f;
+  }
+  } else {
+    // ------------------------------------------------ softmax warpgroups A (warps 4-7) and B (8-11)
+    regs_inc<TR::REGS_HIGH>();
+    const int wg = (warp - 4) >> 2;                // 0 = A, 1 = B
+    const int row = (threadIdx.x - 128) & 127;     // TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tbase + lane_off + TR::S_COL0 + wg * BN;
+    const uint32_t tOA = tbase + lane_off + TR::O_COL0;
+    const uint32_t tOB = tOA + D;
+    const uint32_t tO = wg ? tOB : tOA;
+    const float scale = p.softmax_scale > 0.f ? p.softmax_scale : rsqrtf(static_cast<float>(D));
+    const float sl2 = scale * 1.4426950408889634f;
+    long long it = it_begin;
+    Piece pc;
+    int cnt = 0, pidx = 0;
+    bool ok = true;
+    while (next_piece(it, pc)) {
       float m_run = -INFINITY, l_run = 0.f;
-      bool ok = true;
-      for (int j = 0; j < nkv && ok; ++j) {
-        // tcgen05.ld is warp-collective: every lane must agree before using it
-        if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1, s_abort))) { ok = false; break; }
+      int mine = 0;
+      for (int i = wg; i < pc.n; i += 2, ++mine) {
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], cnt & 1, s_abort));
+        if (!ok) continue;
         tc_fence_after();
-        const uint32_t tS = tbase + lane_off + ((j & 1) ? TR::S_COL1 : TR::S_COL0);
         uint32_t sr[BN / 32][32];
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) tmem_load32(tS + c * 32, sr[c]);
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) tmem_load_wait(sr[c]);
-        const int kv_valid = p.Nk - j * BN;
-        float mx = -INFINITY;
-        if (kv_valid >= BN) {
+        const int kv_valid = p.Nk - (pc.j0 + i) * BN;
+        if (kv_valid < BN) {
 #pragma unroll
           for (int c = 0; c < BN / 32; ++c)
 #pragma unroll
-            for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[c][e]));
-        } else {
-#pragma unroll
-          for (int c = 0; c < BN / 32; ++c)
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
+            for (int e = 0; e < 32; ++e)
               if (c * 32 + e >= kv_valid) sr[c][e] = __float_as_uint(-INFINITY);
-              mx = fmaxf(mx, __uint_as_float(sr[c][e]));
-            }
         }
+        // row max with 8 independent chains (max is exact in any order)
+        float mx8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BN / 32; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(sr[c][e]));
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float m_new = mx * sl2;
         float m_use = m_run;
         bool rescale = false;
         if (m_new > m_run + 8.0f) {
           m_use = m_new;
-          rescale = (j > 0);
+          rescale = (mine > 0);
         }
-        // P buffer and O are free once the previous P V has completed
-        if (j > 0) {
-          if (!__all_sync(0xffffffffu, mbar_wait(o_done, (j - 1) & 1, s_abort))) { ok = false; break; }
-          tc_fence_after();
-        }
-        // tcgen05.ld/st are warp-collective: the warp rescales together when any
-        // of its rows needs it; rows that do not scale by 1
+        // S_i complete implies this warpgroup's previous P V (issued before it) is complete
         if (__any_sync(0xffffffffu, rescale)) {
           const float alpha = rescale ? ex2(m_run - m_use) : 1.0f;
           l_run *= alpha;
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
-            tmem_load32(tbase + lane_off + TR::O_COL + c * 32, o);
+            tmem_load32(tO + c * 32, o);
             tmem_load_wait(o);
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_store32(tbase + lane_off + TR::O_COL + c * 32, o);
+            tmem_store32(tO + c * 32, o);
           }
-          tmem_store_wait();
         }
         m_run = m_use;
         const float neg_m = -m_use;
-        float lsum = 0.f;
-        if constexpr (TR::ES == 2) {
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};  // 4 independent partial sums
 #pragma unroll
-          for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < BN / 32; ++c) {
+          if constexpr (TR::ES == 2) {
+            // packed in place: slot e is written after slots 2e, 2e+1 were read
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {  // 8 probabilities -> one 16-byte chunk
-              float pv[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                pv[e] = ex2(fmaf(__uint_as_float(sr[c][g * 8 + e]), sl2, neg_m));
-                lsum += pv[e];
-              }
-              uint4 u;
-              u.x = pack_bf16(pv[0], pv[1]);
-              u.y = pack_bf16(pv[2], pv[3]);
-              u.z = pack_bf16(pv[4], pv[5]);
-              u.w = pack_bf16(pv[6], pv[7]);
-              const int chunk = c * 4 + g;  // 16-byte chunk index within the P row
-              *reinterpret_cast<uint4*>(sP + (chunk >> 3) * (BM * 128) + sw128_offset(row, chunk & 7)) = u;
+            for (int e = 0; e < 16; ++e) {
+              const float a = ex2(fmaf(__uint_as_float(sr[c][2 * e]), sl2, neg_m));
+              const float a2 = ex2(fmaf(__uint_as_float(sr[c][2 * e + 1]), sl2, neg_m));
+              ls[e & 3] += a + a2;
+              sr[c][e] = pack_bf16(a, a2);
             }
-          }
-        } else {
+            tmem_store16(tS + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[c][0]));
+          } else {
 #pragma unroll
-          for (int c = 0; c < BN / 32; ++c) {
-#pragma unroll
-            for (int g = 0; g < 8; ++g) {  // 4 probabilities -> one 16-byte chunk
-              float pv[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                pv[e] = ex2(fmaf(__uint_as_float(sr[c][g * 4 + e]), sl2, neg_m));
-                lsum += pv[e];
-              }
-              const int chunk = c * 8 + g;
-              *reinterpret_cast<float4*>(sP + (chunk >> 3) * (BM * 128) + sw128_offset(row, chunk & 7)) =
-                  make_float4(pv[0], pv[1], pv[2], pv[3]);
+            for (int e = 0; e < 32; ++e) {
+              const float a = ex2(fmaf(__uint_as_float(sr[c][e]), sl2, neg_m));
+              ls[e & 3] += a;
+              sr[c][e] = __float_as_uint(a);
             }
+            tmem_store32(tS + c * 32, sr[c]);
           }
         }
-        l_run += lsum;
-        fence_proxy_async_smem();
+        l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        tmem_store_wait();
         tc_fence_before();
-        mbar_arrive(p_ready);
+        mbar_arrive(&p_ready[wg]);
+        ++cnt;
       }
-      if (ok && __all_sync(0xffffffffu, mbar_wait(o_done, (nkv - 1) & 1, s_abort))) {
+      // ---- end of the piece: the last P V of this warpgroup must be complete
+      if (mine > 0 && ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_done[wg], (cnt - 1) & 1, s_abort));
+      if (wg == 1) {
+        // B: hand (m, l) over to A once A is done with the previous piece
+        if (pidx > 0 && ok) ok = __all_sync(0xffffffffu, mbar_wait(merged, (pidx - 1) & 1, s_abort));
+        s_mB[row] = mine > 0 ? m_run : -INFINITY;
+        s_lB[row] = mine > 0 ? l_run : 0.f;
+        tc_fence_before();
+        mbar_arrive(b_ready);
+      } else {
+        // A: merge the two halves, then write O (whole unit) or a partial
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(b_ready, pidx & 1, s_abort));
         tc_fence_after();
-        const int t = q0 + row;
-        const float inv_l = 1.0f / l_run;
-        T* out = static_cast<T*>(p.out);
+        const bool hasB = pc.n >= 2;
+        const float mB = s_mB[row], lB = s_lB[row];
+        const float mm = fmaxf(m_run, mB);
+        const float aA = ex2(m_run - mm);
+        const float aB = hasB ? ex2(mB - mm) : 0.f;
+        const float L = l_run * aA + lB * aB;
+        const int qt = pc.u % p.q_tiles;
+        const int h = (pc.u / p.q_tiles) % p.H;
+        const int b = pc.u / (p.q_tiles * p.H);
+        const int t = qt * BM + row;
+        const bool whole = (pc.j0 == 0 && pc.n == p.nkv);
+        const long long first_it = static_cast<long long>(pc.u) * p.nkv;
+        const int g_first = owner_of(first_it, p.total, p.grid);
+        const int g_last = owner_of(first_it + p.nkv - 1, p.total, p.grid);
+        float* slot = p.partials + static_cast<size_t>(g + pc.u) * TR::SLOT_FLOATS;
+        const float inv_L = 1.0f / L;
+        if (ok) {
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_load32(tbase + lane_off + TR::O_COL + c * 32, o);
-          tmem_load_wait(o);
-          if (t < p.Tq) {
-            T* dst = out + ((static_cast<long long>(b) * p.Tq + t) * p.H + h) * D + c * 32;
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t oa[32], ob[32];
+            tmem_load32(tOA + c * 32, oa);
+            tmem_load_wait(oa);
+            if (hasB) {
+              tmem_load32(tOB + c * 32, ob);
+              tmem_load_wait(ob);
+            }
+            float* x = reinterpret_cast<float*>(oa);  // merged in place
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              float x[8];
+            for (int e = 0; e < 32; ++e)
+              x[e] = __uint_as_float(oa[e]) * aA + (hasB ? __uint_as_float(ob[e]) * aB : 0.f);
+            if (whole) {
+              if (t < p.Tq) {
+                T* dst = static_cast<T*>(p.out) + ((static_cast<size_t>(b) * p.Tq + t) * p.H + h) * D + c * 32;
 #pragma unroll
-              for (int e = 0; e < 8; ++e) x[e] = __uint_as_float(o[g * 8 + e]) * inv_l;
-              store_chunk8<T>(dst + g * 8, x);
+                for (int q8 = 0; q8 < 4; ++q8) {
+                  float y[8];
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) y[e] = x[q8 * 8 + e] * inv_L;
+                  store_chunk8<T>(dst + q8 * 8, y);
+                }
+              }
+            } else {
+              float4* dst = reinterpret_cast<float4*>(slot + static_cast<size_t>(row) * D + c * 32);
+#pragma unroll
+              for (int q4 = 0; q4 < 8; ++q4)
+                dst[q4] = make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]);
             }
           }
         }
-        if (p.lse != nullptr && t < p.Tq)
-          p.lse[(static_cast<long long>(b) * p.H + h) * p.Tq + t] = (m_run + log2f(l_run)) * 0.6931471805599453f;
+        tc_fence_before();
+        mbar_arrive(merged);  // O_A, O_B and s_mB / s_lB may be reused
+        if (whole) {
+          if (ok && p.lse != nullptr && t < p.Tq)
+            p.lse[(static_cast<size_t>(b) * p.H + h) * p.Tq + t] = (mm + log2f(L)) * 0.6931471805599453f;
+        } else {
+          if (ok) {
+            slot[BM * D + row] = mm;
+            slot[BM * D + BM + row] = L;
+          }
+          __threadfence();
+          asm volatile("bar.sync 3, 128;" ::: "memory");
+          if (row == 0) {
+            const int old = ok ? atomicAdd(&p.counters[pc.u], 1) : -1;
+            *s_last = (old == g_last - g_first) ? 1 : 0;
+          }
+          asm volatile("bar.sync 3, 128;" ::: "memory");
+          if (*s_last && ok) {
+            // the last piece of this unit to finish: merge every piece of it
+            __threadfence();
+            float mx = -INFINITY;
+            for (int gg = g_first; gg <= g_last; ++gg)
+              mx = fmaxf(mx, __ldcg(p.partials + static_cast<size_t>(gg + pc.u) * TR::SLOT_FLOATS + BM * D + row));
+            float Lt = 0.f;
+            for (int gg = g_first; gg <= g_last; ++gg) {
+              const float* sl = p.partials + static_cast<size_t>(gg + pc.u) * TR::SLOT_FLOATS;
+              Lt += __ldcg(sl + BM * D + BM + row) * ex2(__ldcg(sl + BM * D + row) - mx);
+            }
+            const float inv = 1.0f / Lt;
+#pragma unroll 1
+            for (int c = 0; c < D / 8; ++c) {
+              float y[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) y[e] = 0.f;
+              for (int gg = g_first; gg <= g_last; ++gg) {
+                const float* sl = p.partials + static_cast<size_t>(gg + pc.u) * TR::SLOT_FLOATS;
+                const float a = ex2(__ldcg(sl + BM * D + row) - mx) * inv;
+                const float4 v0 = __ldcg(reinterpret_cast<const float4*>(sl + static_cast<size_t>(row) * D + c * 8));
+                const float4 v1 =
+                    __ldcg(reinterpret_cast<const float4*>(sl + static_cast<size_t>(row) * D + c * 8 + 4));
+                y[0] += v0.x * a; y[1] += v0.y * a; y[2] += v0.z * a; y[3] += v0.w * a;
+                y[4] += v1.x * a; y[5] += v1.y * a; y[6] += v1.z * a; y[7] += v1.w * a;
+              }
+              if (t < p.Tq)
+                store_chunk8<T>(static_cast<T*>(p.out) + ((static_cast<size_t>(b) * p.Tq + t) * p.H + h) * D + c * 8,
+                                y);
+            }
+            if (p.lse != nullptr && t < p.Tq)
+              p.lse[(static_cast<size_t>(b) * p.H + h) * p.Tq + t] = (mx + log2f(Lt)) * 0.6931471805599453f;
+          }
+        }
       }
+      ++pidx;
     }
   }
 

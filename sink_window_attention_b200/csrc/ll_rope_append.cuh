@@ -27,24 +27,26 @@ struct RopeParams {
 
 // omega_i = base^(-2i/d) for pair j = 0..P-1 of head h (P = D/2): the temporal
 // band (j < pt) uses base theta0 (1 + sigma eps_h), the row and column bands
-// theta0; inside a band of `pairs` pairs, d = 2 * pairs.
+// theta0; inside a band of `pairs` pairs, d = 2 * pairs. Evaluated in fp32 as
+// exp2(-(i/pairs) * log2(base)): the relative error of omega is below 1e-6,
+// i.e. under 3e-4 rad of angle at position 3000, far below bf16 resolution.
 __device__ __forceinline__ float omega_of(const RopeParams& rp, int h, int j) {
-  double base;
+  float base;
   int i, pairs;
   if (j < rp.pt) {
-    base = rp.theta0 * (1.0 + rp.sigma * static_cast<double>(rp.eps[h]));
+    base = static_cast<float>(rp.theta0 * (1.0 + rp.sigma * static_cast<double>(rp.eps[h])));
     i = j;
     pairs = rp.pt;
   } else if (j < rp.pt + rp.ph) {
-    base = rp.theta0;
+    base = static_cast<float>(rp.theta0);
     i = j - rp.pt;
     pairs = rp.ph;
   } else {
-    base = rp.theta0;
+    base = static_cast<float>(rp.theta0);
     i = j - rp.pt - rp.ph;
     pairs = rp.pw;
   }
-  return static_cast<float>(exp2(-(static_cast<double>(i) / pairs) * log2(base)));
+  return exp2f(-(static_cast<float>(i) / static_cast<float>(pairs)) * log2f(base));
 }
 
 // omega[hh * P + j] for heads h0 .. h0+nh-1, built by the whole block.
@@ -151,20 +153,21 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(const RopeApplyParams p
   build_omega(s_omega, p.rp, 0, p.H, P);
   __syncthreads();
   const int cpr = p.D / 8;  // chunks per (token, head) row
-  const long long total = static_cast<long long>(p.B) * p.F * p.N * p.H * cpr;
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  const int total = p.B * p.F * p.N * p.H * cpr;  // < 2^31, checked on the host
+  const int FN = p.F * p.N;
   T* x = static_cast<T*>(p.x);
   const int pth = p.rp.pt + p.rp.ph;
-  for (long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total; idx += stride) {
-    const long long row = idx / cpr;
-    const int c = static_cast<int>(idx - row * cpr);
-    const int h = static_cast<int>(row % p.H);
-    const long long tok = (row / p.H) % (static_cast<long long>(p.F) * p.N);
-    const int fi = static_cast<int>(tok / p.N);
-    const int n = static_cast<int>(tok - static_cast<long long>(fi) * p.N);
+  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += gridDim.x * blockDim.x) {
+    const int row = idx / cpr;
+    const int c = idx - row * cpr;
+    const int bt = row / p.H;
+    const int h = row - bt * p.H;
+    const int tok = bt % FN;
+    const int fi = tok / p.N;
+    const int n = tok - fi * p.N;
     const int r = n / p.rp.grid_w, col = n - r * p.rp.grid_w;
     float v[8];
-    T* ptr = x + row * p.D + c * 8;
+    T* ptr = x + static_cast<size_t>(row) * p.D + c * 8;
     load_chunk8<T>(ptr, v);
     rotate_chunk8(v, c * 4, static_cast<float>(p.rp.t_first + fi), static_cast<float>(r),
                   static_cast<float>(col), s_omega + h * P, p.rp.pt, pth);
@@ -204,33 +207,32 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
   if (p.rp.enabled) build_omega(s_omega, p.rp, 0, p.H, P);
   __syncthreads();
   const int cpr = p.D / 8;
-  const long long total = static_cast<long long>(p.B) * p.F * p.N * p.H * cpr;
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  const int total = p.B * p.F * p.N * p.H * cpr;  // < 2^31, checked on the host
+  const int FN = p.F * p.N;
+  const int S = p.n_sink + p.n_local;
   const int pth = p.rp.pt + p.rp.ph;
   const Tin* kin = static_cast<const Tin*>(p.k_in);
   const Tin* vin = static_cast<const Tin*>(p.v_in);
   // All threads of the block run the same number of iterations, so the
   // shuffles of the FP8 path always see full warps.
-  for (long long base = static_cast<long long>(blockIdx.x) * blockDim.x; base < total; base += stride) {
-    const long long idx = base + threadIdx.x;
+  for (int base = blockIdx.x * blockDim.x; base < total; base += gridDim.x * blockDim.x) {
+    const int idx = base + threadIdx.x;
     const bool active = idx < total;
-    const long long i = active ? idx : 0;
-    const long long row = i / cpr;
-    const int c = static_cast<int>(i - row * cpr);
-    const int h = static_cast<int>(row % p.H);
-    const long long bt = row / p.H;                         // b * F*N + tok
-    const long long FN = static_cast<long long>(p.F) * p.N;
-    const int b = static_cast<int>(bt / FN);
-    const long long tok = bt - b * FN;
-    const int fi = static_cast<int>(tok / p.N);
-    const int n = static_cast<int>(tok - static_cast<long long>(fi) * p.N);
-    const int S = p.n_sink + p.n_local;
+    const int i = active ? idx : 0;
+    const int row = i / cpr;
+    const int c = i - row * cpr;
+    const int bt = row / p.H;                       // b * F*N + tok
+    const int h = row - bt * p.H;
+    const int b = bt / FN;
+    const int tok = bt - b * FN;
+    const int fi = tok / p.N;
+    const int n = tok - fi * p.N;
     const int slot = cache_slot(p.first_frame + fi, p.n_sink, p.n_local);
-    const long long drow = (static_cast<long long>(b) * S * p.N + static_cast<long long>(slot) * p.N + n) * p.H + h;
+    const size_t drow = (static_cast<size_t>(b) * S * p.N + static_cast<size_t>(slot) * p.N + n) * p.H + h;
     float kx[8], vx[8];
     if (active) {
-      load_chunk8<Tin>(kin + row * p.D + c * 8, kx);
-      load_chunk8<Tin>(vin + row * p.D + c * 8, vx);
+      load_chunk8<Tin>(kin + static_cast<size_t>(row) * p.D + c * 8, kx);
+      load_chunk8<Tin>(vin + static_cast<size_t>(row) * p.D + c * 8, vx);
       if (p.rp.enabled) {
         const int r = n / p.rp.grid_w, col = n - r * p.rp.grid_w;
         rotate_chunk8(kx, c * 4, static_cast<float>(p.rp.t_first + fi), static_cast<float>(r),
