@@ -14,9 +14,11 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  * - All tensor pointers are DEVICE pointers into caller-owned memory unless a
- *   parameter says "host". The library never allocates device memory and keeps
- *   no state between calls; every call is asynchronous on `stream`
- *   (a cudaStream_t passed as void*, NULL = legacy default stream).
+ *   parameter says "host". No call allocates device memory and no call keeps
+ *   state for the next one (the one device buffer the library owns is the
+ *   static scratch array of ll_sink_window_attention_noalloc); every call is
+ *   asynchronous on `stream` (a cudaStream_t passed as void*, NULL = legacy
+ *   default stream).
  * - Token tensors use the layout [B][T][H][D] (row-major, D fastest), with
  *   T = frames * N, N = grid_h * grid_w tokens per latent frame in row-major
  *   (grid row, grid column) order.
@@ -176,6 +178,35 @@ ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvc
                                    const ll_rope_desc* rope, float softmax_scale,
                                    void* out, float* lse, void* workspace,
                                    size_t workspace_bytes, void* stream);
+
+/*
+ * Allocation-free variant of ll_sink_window_attention (the pages have no
+ * counterpart; this is a library convenience).
+ * Some callers cannot call cudaMalloc or any allocating routine: cudaMalloc
+ * may synchronise the whole device, which a frame-rate loop cannot afford,
+ * and plugin hosts that own all device memory through their own pools forbid
+ * allocation outside them. This entry point takes the same arguments minus
+ * the workspace and uses instead a scratch array of
+ * LL_NOALLOC_SCRATCH_BYTES bytes that the library holds in static device
+ * memory: every GPU that loads the library keeps it until the process exits.
+ * - The first call on a device looks up that device's copy of the array (with
+ *   the device current); make that first call before any stream capture.
+ * - Requests whose scratch need, ll_sink_window_attention_workspace_bytes(),
+ *   exceeds LL_NOALLOC_SCRATCH_BYTES are rejected with LL_ERR_INVALID_ARG
+ *   before anything is launched.
+ * - All calls on a device share the one array and it keeps the contents of
+ *   the last call (the parts that must start at zero are cleared by each
+ *   call); calls that overlap on the GPU (e.g. on two streams without
+ *   ordering between them) race and give undefined results.
+ * - It allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * Other arguments, layouts and errors as for ll_sink_window_attention.
+ */
+#define LL_NOALLOC_SCRATCH_BYTES (48u * 1024u * 1024u)
+
+ll_status ll_sink_window_attention_noalloc(const void* q, ll_dtype q_dtype, const ll_kvcache* cache,
+                                           long long first_frame, int n_query_frames,
+                                           const ll_rope_desc* rope, float softmax_scale, void* out,
+                                           float* lse, void* stream);
 
 /*
  * KV recache at a prompt switch (LongLive review, "KV Recache": the cache is

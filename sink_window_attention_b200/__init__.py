@@ -25,8 +25,9 @@ MAX_HEADS = 64
 EXPORTED = (
     "ll_abi_version", "ll_last_error", "ll_slot_of_frame", "ll_device_error", "ll_rope_apply",
     "ll_kvcache_append", "ll_sink_window_attention_workspace_bytes", "ll_sink_window_attention",
-    "ll_kv_recache_workspace_bytes", "ll_kv_recache",
+    "ll_kv_recache_workspace_bytes", "ll_kv_recache", "ll_sink_window_attention_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 48 * 1024 * 1024
 
 
 class LLError(RuntimeError):
@@ -70,6 +71,7 @@ def lib() -> ctypes.CDLL:
         L.ll_sink_window_attention_workspace_bytes.argtypes = [cp, i]
         L.ll_sink_window_attention_workspace_bytes.restype = sz
         L.ll_sink_window_attention.argtypes = [vp, i, cp, ll_, i, rp, f, vp, vp, vp, sz, vp]
+        L.ll_sink_window_attention_noalloc.argtypes = [vp, i, cp, ll_, i, rp, f, vp, vp, vp]
         L.ll_kv_recache_workspace_bytes.argtypes = [cp, i, i]
         L.ll_kv_recache_workspace_bytes.restype = sz
         L.ll_kv_recache.argtypes = [cp, vp, i, vp, vp, vp, f, ctypes.POINTER(ll_), i, rp, vp, sz, vp]
@@ -243,6 +245,20 @@ def sink_window_attention(q: torch.Tensor, cache: KVCache, first_frame: int, rop
     _check(lib().ll_sink_window_attention(_ptr(q), _dtype_code(q.dtype), ctypes.byref(cache.to_c()), first_frame, F,
                                           _rope_ref(rope), float(softmax_scale), _ptr(out), _ptr(lse),
                                           _ptr(workspace), ws_bytes, _stream(stream)))
+    return out
+
+
+def sink_window_attention_noalloc(q: torch.Tensor, cache: KVCache, first_frame: int, rope: Optional[Rope],
+                                  softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                                  lse: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """ll_sink_window_attention_noalloc: the same attention with the library's
+    static scratch array instead of a caller workspace (allocates nothing)."""
+    F = q.shape[1] // cache.N
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().ll_sink_window_attention_noalloc(_ptr(q), _dtype_code(q.dtype), ctypes.byref(cache.to_c()),
+                                                  first_frame, F, _rope_ref(rope), float(softmax_scale), _ptr(out),
+                                                  _ptr(lse), _stream(stream)))
     return out
 
 

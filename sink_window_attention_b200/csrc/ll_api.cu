@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "../../include/ll_api.h"
@@ -352,6 +353,57 @@ ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvc
   if (f32 && cache->D == 64)
     return launch_attention<ll::AttnTraits<64, float>>(p, cache, S, workspace, workspace_bytes, s);
   return fail(LL_ERR_UNSUPPORTED, "attention supports D = 64 or 128 (bf16) and D = 64 (f32); got D = %d", cache->D);
+}
+
+}  // extern "C"
+
+// Scratch of ll_sink_window_attention_noalloc: one copy per device that loads
+// the library, alive until the process exits. In host code the symbol is only
+// a handle; its device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LL_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the current device's scratch array (looked up once per
+// device, with that device current).
+ll_status noalloc_scratch(void** ptr) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return check_launch("cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(LL_ERR_UNSUPPORTED, "device ordinal %d is out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(LL_ERR_CUDA, "cudaGetSymbolAddress(scratch) failed: %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *ptr = g_noalloc_ptr[dev];
+  return LL_OK;
+}
+}  // namespace
+
+extern "C" {
+
+ll_status ll_sink_window_attention_noalloc(const void* q, ll_dtype q_dtype, const ll_kvcache* cache,
+                                           long long first_frame, int n_query_frames, const ll_rope_desc* rope,
+                                           float softmax_scale, void* out, float* lse, void* stream) {
+  g_last_error.clear();
+  if (cache == nullptr) return fail(LL_ERR_INVALID_ARG, "cache is NULL");
+  const size_t need = ll_sink_window_attention_workspace_bytes(cache, n_query_frames);
+  if (need > LL_NOALLOC_SCRATCH_BYTES)
+    return fail(LL_ERR_INVALID_ARG,
+                "this call needs %zu bytes of scratch; the static scratch array holds %u "
+                "(use ll_sink_window_attention with a caller workspace)",
+                need, LL_NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  const ll_status st = noalloc_scratch(&scratch);
+  if (st != LL_OK) return st;
+  return ll_sink_window_attention(q, q_dtype, cache, first_frame, n_query_frames, rope, softmax_scale, out, lse,
+                                  scratch, LL_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 size_t ll_kv_recache_workspace_bytes(const ll_kvcache* cache, int d_model, int n_slots) {

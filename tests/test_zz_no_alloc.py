@@ -1,0 +1,65 @@
+"""The allocation-free attention entry point, ll_sink_window_attention_noalloc.
+
+It is for callers that cannot call cudaMalloc (it may synchronise the whole
+device, which a frame-rate loop cannot afford; plugin hosts that own all device
+memory forbid allocation outside their pools). It runs the same attention with
+the library's static scratch array instead of a caller workspace. This file is
+collected last so that a run stopping at the first failure has run every other
+test before it; it also passes on its own in a fresh process.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import sink_window_attention_b200 as swa
+import swa_workloads as W
+from tests.conftest import assert_parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from sink_window_attention_b200 import build
+    build.build()
+    swa.lib()
+
+
+def test_noalloc_matches_workspace_entry_point():
+    w = W.WAN
+    eps = W.jitter_eps(4, w.H)
+    rope = swa.Rope(pairs=w.pairs, grid_h=w.grid_h, grid_w=w.grid_w, theta0=w.theta0, sigma_t=0.8,
+                    eps=[float(e) for e in eps])
+    cache = swa.KVCache(1, w.H, w.D, w.N, "bf16")
+    for f in range(12):
+        _, k, v = W.qkv_frames(w, 5, f, 1, device="cuda")
+        swa.kvcache_append(cache, k, v, f, rope)
+    for f in (12, 13):
+        q, k, v = W.qkv_frames(w, 5, f, 1, device="cuda")
+        swa.kvcache_append(cache, k, v, f, rope)
+        lse_ref = torch.empty(1, w.H, w.N, device="cuda")
+        ref = swa.sink_window_attention(q, cache, f, rope, lse=lse_ref)
+        # two calls in a row on the shared static scratch
+        for _ in range(2):
+            lse = torch.empty_like(lse_ref)
+            out = swa.sink_window_attention_noalloc(q, cache, f, rope, lse=lse)
+            torch.cuda.synchronize()
+            assert_parity(out.double().cpu().numpy(), ref.double().cpu().numpy(), what=f"noalloc frame {f}")
+            assert_parity(lse.cpu().numpy(), lse_ref.cpu().numpy(), max_rel=1e-3, mean_abs=5e-3, what="lse")
+    assert swa.device_error() == 0
+
+
+def test_noalloc_rejects_requests_beyond_the_static_scratch():
+    c = swa.KVCacheC()
+    c.k, c.v = 4096, 8192            # never dereferenced: the size check comes first
+    c.k_scale = c.v_scale = None
+    c.dtype, c.B, c.H, c.D = swa.LL_BF16, 8, 64, 128
+    c.tokens_per_frame, c.n_sink, c.n_local = 1560, 3, 9
+    need = swa.lib().ll_sink_window_attention_workspace_bytes(ctypes.byref(c), 1)
+    assert need > swa.NOALLOC_SCRATCH_BYTES
+    st = swa.lib().ll_sink_window_attention_noalloc(1 << 20, swa.LL_BF16, ctypes.byref(c), 20, 1, None, 0.0,
+                                                    1 << 21, None, None)
+    assert st == swa.LL_ERR_INVALID_ARG
+    assert "static scratch" in swa.last_error()
