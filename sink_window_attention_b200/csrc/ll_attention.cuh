@@ -58,6 +58,7 @@ struct AttnTraits {
   static constexpr int MMA_K = 32 / ES;             // reduction elements per MMA
   static constexpr int FMT = (ES == 2) ? 1 : 2;     // bf16 / tf32
   static constexpr int QST = 2;                     // Q buffers
+  static constexpr int EXP_FMA_FROM = 8;            // pairs e with (e % 8) >= this use exp2_fma_x2 (8: none)
   static constexpr int CTRL_BYTES = 2048;
   static constexpr int STAGE_BUDGET = 232448 - CTRL_BYTES - 1024 - QST * Q_BYTES;
   static constexpr int STAGES = STAGE_BUDGET / KV_BYTES;
@@ -110,7 +111,7 @@ __device__ __forceinline__ int owner_of(long long i, long long total, int G) {
 
 // Q tile of unit u, rotated with this head's frequencies `om` [D/2], into
 // the 128-byte-swizzled K-major operand layout at sQ.
-template <class TR>
+template <class TR, int BATCH>
 __device__ __forceinline__ void load_q_tile(uint8_t* sQ, const AttnParams& p, const float* om, int u, int tid,
                                             int nthreads) {
   using T = typename TR::T;
@@ -121,37 +122,49 @@ __device__ __forceinline__ void load_q_tile(uint8_t* sQ, const AttnParams& p, co
   const int q0 = qt * BM;
   const T* q = static_cast<const T*>(p.q);
   constexpr int GPR = D / 8;  // 8-element groups per row
+  // BATCH global loads in flight per thread
   const int pth = p.rp.pt + p.rp.ph;
-  for (int g = tid; g < BM * GPR; g += nthreads) {
-    const int r = g / GPR, e8 = g - r * GPR;
-    const int t = q0 + r;
-    float x[8];
-    if (t < p.Tq) {
-      load_chunk8<T>(q + ((static_cast<size_t>(b) * p.Tq + t) * p.H + h) * D + e8 * 8, x);
-      if (p.rp.enabled) {
+  for (int g0 = tid; g0 < BM * GPR; g0 += BATCH * nthreads) {
+    float x[BATCH][8];
+#pragma unroll
+    for (int k = 0; k < BATCH; ++k) {
+      const int g = g0 + k * nthreads;
+      const int r = g / GPR, e8 = g - r * GPR;
+      const int t = q0 + r;
+      if (g < BM * GPR && t < p.Tq) {
+        load_chunk8<T>(q + ((static_cast<size_t>(b) * p.Tq + t) * p.H + h) * D + e8 * 8, x[k]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[k][i] = 0.f;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < BATCH; ++k) {
+      const int g = g0 + k * nthreads;
+      if (g >= BM * GPR) break;
+      const int r = g / GPR, e8 = g - r * GPR;
+      const int t = q0 + r;
+      if (p.rp.enabled && t < p.Tq) {
         const int fi = t / p.N, n = t - fi * p.N;
         const int rr = n / p.rp.grid_w, cc = n - rr * p.rp.grid_w;
-        rotate_chunk8(x, e8 * 4, static_cast<float>(p.rp.t_first + fi), static_cast<float>(rr),
+        rotate_chunk8(x[k], e8 * 4, static_cast<float>(p.rp.t_first + fi), static_cast<float>(rr),
                       static_cast<float>(cc), om, p.rp.pt, pth);
       }
-    } else {
+      if constexpr (TR::ES == 2) {
+        const int chunk = e8;  // 8 bf16 = 16 bytes
+        uint4 v;
+        v.x = pack_bf16(x[k][0], x[k][1]);
+        v.y = pack_bf16(x[k][2], x[k][3]);
+        v.z = pack_bf16(x[k][4], x[k][5]);
+        v.w = pack_bf16(x[k][6], x[k][7]);
+        *reinterpret_cast<uint4*>(sQ + (chunk >> 3) * (BM * 128) + sw128_offset(r, chunk & 7)) = v;
+      } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] = 0.f;
-    }
-    if constexpr (TR::ES == 2) {
-      const int chunk = e8;  // 8 bf16 = 16 bytes
-      uint4 v;
-      v.x = pack_bf16(x[0], x[1]);
-      v.y = pack_bf16(x[2], x[3]);
-      v.z = pack_bf16(x[4], x[5]);
-      v.w = pack_bf16(x[6], x[7]);
-      *reinterpret_cast<uint4*>(sQ + (chunk >> 3) * (BM * 128) + sw128_offset(r, chunk & 7)) = v;
-    } else {
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int chunk = e8 * 2 + hh;  // 4 floats = 16 bytes
-        *reinterpret_cast<float4*>(sQ + (chunk >> 3) * (BM * 128) + sw128_offset(r, chunk & 7)) =
-            make_float4(x[4 * hh], x[4 * hh + 1], x[4 * hh + 2], x[4 * hh + 3]);
+        for (int hh = 0; hh < 2; ++hh) {
+          const int chunk = e8 * 2 + hh;  // 4 floats = 16 bytes
+          *reinterpret_cast<float4*>(sQ + (chunk >> 3) * (BM * 128) + sw128_offset(r, chunk & 7)) =
+              make_float4(x[k][4 * hh], x[k][4 * hh + 1], x[k][4 * hh + 2], x[k][4 * hh + 3]);
+        }
       }
     }
   }
@@ -185,9 +198,9 @@ __global__ void __launch_bounds__(384, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   volatile int* s_last = reinterpret_cast<volatile int*>(s_tmem + 2);
-  float* s_mB = reinterpret_cast<float*>(ctrl + 256);      // [128]
+  float* s_mB = reinterpret_cast<float*>(ctrl + 384);      // [128]
   float* s_lB = s_mB + BM;                                 // [128]
-  float* s_omega = reinterpret_cast<float*>(ctrl + 1280);  // [2][D/2]: one head per Q buffer
+  float* s_omega = reinterpret_cast<float*>(ctrl + 1408);  // [2][D/2]: one head per Q buffer
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.x;
@@ -235,6 +248,23 @@ __global__ void __launch_bounds__(384, 1)
     it += pc.n;
     return true;
   };
+
+  // The first piece's Q is loaded by warps 2-11 together (the softmax
+  // warpgroups have nothing to do before it); later pieces by warps 2-3.
+  {
+    long long it0 = it_begin;
+    Piece pc0;
+    next_piece(it0, pc0);
+    if (warp >= 2) {
+      const int tid = threadIdx.x - 64;  // 0..319
+      if (p.rp.enabled)
+        for (int j = tid; j < D / 2; j += 320) s_omega[j] = omega_of(p.rp, (pc0.u / p.q_tiles) % p.H, j);
+      asm volatile("bar.sync 4, 320;" ::: "memory");
+      load_q_tile<TR, 4>(sQ, p, s_omega, pc0.u, tid, 320);
+      asm volatile("bar.sync 4, 320;" ::: "memory");
+      if (tid == 0) mbar_arrive(&q_full[0]);
+    }
+  }
 
   if (warp < 4) {
   // warpgroup 0: producer, MMA issuer, Q loader (same setmaxnreg for its four warps)
@@ -295,17 +325,22 @@ __global__ void __launch_bounds__(384, 1)
       Piece pc;
       int kc = 0, vc = 0, pidx = 0;
       bool ok = true;
+      // descriptor words of every buffer, computed once; an MMA then only adds
+      // a constant to the low word
+      const DescWords dQ = desc_words(aQ, 16, 1024, 2), dK = desc_words(aK, 16, 1024, 2);
+      const DescWords dV = TR::ES == 2 ? desc_words(aV, BN * 128, 1024, 2) : desc_words(aV, BN * 128, 512, 1);
       auto issue_s = [&](int w, int qb) -> bool {
         const int st = kc % KST;
         if (!mbar_wait(&k_full[st], (kc / KST) & 1, s_abort)) return false;
         tc_fence_after();
         const uint32_t d = tbase + TR::S_COL0 + w * BN;
+        const uint32_t qoff = qb * TR::Q_BYTES, koff = st * TR::KV_BYTES;
 #pragma unroll
         for (int k = 0; k < TR::QK_STEPS; ++k) {
           const uint32_t off = (k >> 2) * (BM * 128) + (k & 3) * 32;
           const uint32_t offk = (k >> 2) * (BN * 128) + (k & 3) * 32;
-          const uint64_t da = desc_sw128(aQ + qb * TR::Q_BYTES + off, 16, 1024);
-          const uint64_t db = desc_sw128(aK + st * TR::KV_BYTES + offk, 16, 1024);
+          const uint64_t da = desc_at(dQ, qoff + off);
+          const uint64_t db = desc_at(dK, koff + offk);
           if constexpr (TR::ES == 2) mma_bf16_ss(d, da, db, idS, k > 0 ? 1u : 0u);
           else mma_tf32_ss(d, da, db, idS, k > 0 ? 1u : 0u);
         }
@@ -314,25 +349,20 @@ __global__ void __launch_bounds__(384, 1)
         ++kc;
         return true;
       };
-      auto issue_pv = [&](int w, bool acc) -> bool {
+      auto issue_pv = [&](int w, bool acc) {
         const int st = vc % VST;
-        if (!mbar_wait(&v_full[st], (vc / VST) & 1, s_abort)) return false;
-        tc_fence_after();
         const uint32_t d = tbase + TR::O_COL0 + w * D;
         const uint32_t pa = tbase + TR::S_COL0 + w * BN;  // P_w aliases S_w
+        const uint32_t voff = st * TR::KV_BYTES;
 #pragma unroll
         for (int k = 0; k < TR::PV_STEPS; ++k) {
-          const uint32_t av = aV + st * TR::KV_BYTES + k * TR::MMA_K * 128;
-          if constexpr (TR::ES == 2) {
-            mma_bf16_ts(d, pa + k * 8, desc_sw128(av, BN * 128, 1024), idO, (acc || k > 0) ? 1u : 0u);
-          } else {
-            mma_tf32_ts(d, pa + k * 8, desc_mn_sw128_atom32(av, BN * 128, 512), idO, (acc || k > 0) ? 1u : 0u);
-          }
+          const uint64_t db = desc_at(dV, voff + k * TR::MMA_K * 128);
+          if constexpr (TR::ES == 2) mma_bf16_ts(d, pa + k * 8, db, idO, (acc || k > 0) ? 1u : 0u);
+          else mma_tf32_ts(d, pa + k * 8, db, idO, (acc || k > 0) ? 1u : 0u);
         }
         mma_commit(&o_done[w]);
         mma_commit(&v_empty[st]);
         ++vc;
-        return true;
       };
       int pcnt[2] = {0, 0};  // P tiles consumed per softmax warpgroup
       while (ok && next_piece(it, pc)) {
@@ -345,8 +375,9 @@ __global__ void __launch_bounds__(384, 1)
           ++pcnt[w];
           // the previous piece's O_A / O_B must have been read before the first P V overwrites them
           if (i == 0 && pidx > 0 && !mbar_wait(merged, (pidx - 1) & 1, s_abort)) { ok = false; break; }
+          if (!mbar_wait(&v_full[vc % VST], (vc / VST) & 1, s_abort)) { ok = false; break; }
           tc_fence_after();
-          if (!issue_pv(w, i >= 2)) { ok = false; break; }
+          issue_pv(w, i >= 2);
           if (i + 2 < pc.n && !issue_s(w, qb)) { ok = false; break; }
         }
         mma_commit(&q_empty[qb]);  // Q buffer free once every MMA issued so far has completed
@@ -360,7 +391,8 @@ __global__ void __launch_bounds__(384, 1)
     const int tid = threadIdx.x - 64;  // 0..63
     long long it = it_begin;
     Piece pc;
-    int pidx = 0;
+    next_piece(it, pc);  // the first piece was loaded above
+    int pidx = 1;
     while (next_piece(it, pc)) {
       const int qb = pidx & 1;
       const int h = (pc.u / p.q_tiles) % p.H;
@@ -369,7 +401,7 @@ __global__ void __launch_bounds__(384, 1)
       if (ok && p.rp.enabled)
         for (int j = tid; j < D / 2; j += 64) om[j] = omega_of(p.rp, h, j);
       asm volatile("bar.sync 2, 64;" ::: "memory");
-      if (ok) load_q_tile<TR>(sQ + qb * TR::Q_BYTES, p, om, pc.u, tid, 64);
+      if (ok) load_q_tile<TR, 2>(sQ + qb * TR::Q_BYTES, p, om, pc.u, tid, 64);
       asm volatile("bar.sync 2, 64;" ::: "memory");
       if (tid == 0) mbar_arrive(&q_full[qb]);
       ++pidx;
@@ -399,28 +431,40 @@ __global__ void __launch_bounds__(384, 1)
         if (!ok) continue;
         tc_fence_after();
         uint32_t sr[BN / 32][32];
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) tmem_load32(tS + c * 32, sr[c]);
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) tmem_load_wait(sr[c]);
+        constexpr int HC = BN / 64;  // chunks of 32 columns per half
         const int kv_valid = p.Nk - (pc.j0 + i) * BN;
-        if (kv_valid < BN) {
-#pragma unroll
-          for (int c = 0; c < BN / 32; ++c)
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (c * 32 + e >= kv_valid) sr[c][e] = __float_as_uint(-INFINITY);
-        }
-        // row max with 8 independent chains (max is exact in any order)
+        // row max: 3-input max over 8 independent chains (exact in any order);
+        // the second half of S is loaded while the first half is reduced
         float mx8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c)
+        for (int c = 0; c < HC; ++c) tmem_load32(tS + c * 32, sr[c]);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(sr[c][e]));
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int c = 0; c < HC; ++c) tmem_load_wait(sr[c]);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          if (hf == 0) {
+#pragma unroll
+            for (int c = HC; c < 2 * HC; ++c) tmem_load32(tS + c * 32, sr[c]);
+          } else {
+#pragma unroll
+            for (int c = HC; c < 2 * HC; ++c) tmem_load_wait(sr[c]);
+          }
+          if (kv_valid < BN) {
+#pragma unroll
+            for (int c = hf * HC; c < (hf + 1) * HC; ++c)
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (c * 32 + e >= kv_valid) sr[c][e] = __float_as_uint(-INFINITY);
+          }
+#pragma unroll
+          for (int c = hf * HC; c < (hf + 1) * HC; ++c)
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              mx8[e & 7] = fmax3(mx8[e & 7], __uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1]));
+        }
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
         const float m_new = mx * sl2;
         float m_use = m_run;
         bool rescale = false;
@@ -443,31 +487,43 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         m_run = m_use;
-        const float neg_m = -m_use;
-        float ls[4] = {0.f, 0.f, 0.f, 0.f};  // 4 independent partial sums
+        // p = 2^(s * scale * log2(e) - m) on pairs: the argument with one packed
+        // FMA, the exponential on the MUFU unit (optionally some pairs on the FMA
+        // pipe), the running sum in 4 packed partial sums
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_use, -m_use);
+        uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
-          if constexpr (TR::ES == 2) {
-            // packed in place: slot e is written after slots 2e, 2e+1 were read
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float a = ex2(fmaf(__uint_as_float(sr[c][2 * e]), sl2, neg_m));
-              const float a2 = ex2(fmaf(__uint_as_float(sr[c][2 * e + 1]), sl2, neg_m));
-              ls[e & 3] += a + a2;
-              sr[c][e] = pack_bf16(a, a2);
+          for (int e = 0; e < 16; ++e) {
+            const uint64_t x2 =
+                f2_fma(f2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])), sl2x2, negm2);
+            float a, a2;
+            if (TR::EXP_FMA_FROM < 8 && (e & 7) >= TR::EXP_FMA_FROM) {
+              exp2_fma_x2(x2, a, a2);
+            } else {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              a = ex2(x0);
+              a2 = ex2(x1);
             }
-            tmem_store16(tS + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[c][0]));
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float a = ex2(fmaf(__uint_as_float(sr[c][e]), sl2, neg_m));
-              ls[e & 3] += a;
-              sr[c][e] = __float_as_uint(a);
+            ls2[e & 3] = f2_add(ls2[e & 3], f2_pack(a, a2));
+            if constexpr (TR::ES == 2) {
+              sr[c][e] = pack_bf16(a, a2);  // packed in place: slot e is free once 2e, 2e+1 were read
+            } else {
+              sr[c][2 * e] = __float_as_uint(a);
+              sr[c][2 * e + 1] = __float_as_uint(a2);
             }
-            tmem_store32(tS + c * 32, sr[c]);
           }
+          if constexpr (TR::ES == 2) tmem_store16(tS + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[c][0]));
+          else tmem_store32(tS + c * 32, sr[c]);
         }
-        l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        {
+          const uint64_t s01 = f2_add(f2_add(ls2[0], ls2[1]), f2_add(ls2[2], ls2[3]));
+          float u0, u1;
+          f2_unpack(s01, u0, u1);
+          l_run += u0 + u1;
+        }
         tmem_store_wait();
         tc_fence_before();
         mbar_arrive(&p_ready[wg]);
@@ -504,23 +560,23 @@ __global__ void __launch_bounds__(384, 1)
         const float inv_L = 1.0f / L;
         if (ok) {
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t oa[32], ob[32];
-            tmem_load32(tOA + c * 32, oa);
-            tmem_load_wait(oa);
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t oa[16], ob[16];
+            tmem_load16(tOA + c * 16, oa);
+            tmem_load_wait16(oa);
             if (hasB) {
-              tmem_load32(tOB + c * 32, ob);
-              tmem_load_wait(ob);
+              tmem_load16(tOB + c * 16, ob);
+              tmem_load_wait16(ob);
             }
             float* x = reinterpret_cast<float*>(oa);  // merged in place
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
+            for (int e = 0; e < 16; ++e)
               x[e] = __uint_as_float(oa[e]) * aA + (hasB ? __uint_as_float(ob[e]) * aB : 0.f);
             if (whole) {
               if (t < p.Tq) {
-                T* dst = static_cast<T*>(p.out) + ((static_cast<size_t>(b) * p.Tq + t) * p.H + h) * D + c * 32;
+                T* dst = static_cast<T*>(p.out) + ((static_cast<size_t>(b) * p.Tq + t) * p.H + h) * D + c * 16;
 #pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
+                for (int q8 = 0; q8 < 2; ++q8) {
                   float y[8];
 #pragma unroll
                   for (int e = 0; e < 8; ++e) y[e] = x[q8 * 8 + e] * inv_L;
@@ -528,9 +584,9 @@ __global__ void __launch_bounds__(384, 1)
                 }
               }
             } else {
-              float4* dst = reinterpret_cast<float4*>(slot + static_cast<size_t>(row) * D + c * 32);
+              float4* dst = reinterpret_cast<float4*>(slot + static_cast<size_t>(row) * D + c * 16);
 #pragma unroll
-              for (int q4 = 0; q4 < 8; ++q4)
+              for (int q4 = 0; q4 < 4; ++q4)
                 dst[q4] = make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]);
             }
           }

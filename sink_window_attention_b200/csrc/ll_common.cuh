@@ -72,6 +72,37 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Same contract as mbar_wait, polling with the non-suspending test_wait: for
+// a single latency-critical thread that must react as soon as the phase
+// completes.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const uint32_t a = smem_addr(bar);
+  if (mbar_test(a, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+      if (mbar_test(a, parity)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      atomicOr(&g_error_word, kErrWaitTimeout);
+      *abort = 1;
+      return false;
+    }
+  }
+}
+
 // Bounded wait used during teardown after an abort: ignores the abort flag.
 __device__ __forceinline__ bool mbar_wait_teardown(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_addr(bar);
@@ -173,6 +204,24 @@ __device__ __forceinline__ void tmem_load_wait(uint32_t (&r)[32]) {
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_load16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_load_wait16(uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;\n\t"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+      :
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_store32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -262,6 +311,22 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uin
   return d;
 }
 
+// The two 32-bit words of a descriptor, so that issue loops only add an
+// offset (encoded >> 4) to the low word: addresses below 256 KB never carry
+// out of its 14-bit address field.
+struct DescWords {
+  uint32_t lo, hi;
+};
+__device__ __forceinline__ DescWords desc_words(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+  DescWords w;
+  w.lo = ((saddr & 0x3FFFFu) >> 4) | (((lbo >> 4) & 0x3FFFu) << 16);
+  w.hi = ((sbo >> 4) & 0x3FFFu) | (1u << 14) | (layout << 29);
+  return w;
+}
+__device__ __forceinline__ uint64_t desc_at(DescWords w, uint32_t byte_offset) {
+  return (static_cast<uint64_t>(w.hi) << 32) | (w.lo + (byte_offset >> 4));
+}
+
 // MN-major operand of 32-bit elements (tf32): the only layout the tensor core
 // accepts is the 128-byte swizzle with 32-byte atoms (what a TMA load with
 // CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B writes: 32-byte chunk c of 128-byte row r
@@ -310,6 +375,60 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Packed fp32 pairs (two lanes of one 64-bit register) for the f32x2 FMA-pipe
+// instructions of sm_100.
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for two values on the FMA pipe instead of the MUFU unit.
+// Range reduction x = n + f with n = rint(x), taken with the 1.5 * 2^23
+// rounding constant (the sum's ulp is 1), and f in [-1/2, 1/2]; 2^f by a
+// cubic whose coefficients were fitted for minimal relative error on
+// [-1/2, 1/2] with Lawson's iteratively reweighted least squares (max
+// relative error 7.5e-5 with fp32 Horner evaluation, below the 2^-9 of the
+// bf16 P it feeds); n is then added to the exponent field. x is clamped at
+// -125 so every result is a normal number (2^-125 stands in for smaller
+// values, including -inf).
+__device__ __forceinline__ void exp2_fma_x2(uint64_t x, float& r0, float& r1) {
+  float x0, x1;
+  f2_unpack(x, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t t = f2_add(xc, f2_pack(12582912.0f, 12582912.0f));
+  const uint64_t j = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
+  const uint64_t f = f2_fma(j, f2_pack(-1.0f, -1.0f), xc);
+  uint64_t p = f2_fma(f2_pack(0.0551716685295105f, 0.0551716685295105f), f,
+                      f2_pack(0.2426111400127411f, 0.2426111400127411f));
+  p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
