@@ -2,9 +2,11 @@
 
 Workload (one "step"): one 40-frame prompt segment of the 240 s stream —
 30 attention layers, H=12, D=128, 1560 tokens per latent frame (30x52 grid),
-3 sink + 9 local frames, LoL jitter sigma=0.8 — in steady state: for each of
+3 sink + 9 local frames, LoL jitter sigma=0.8 — in steady state: the segment
+opens with a prompt switch (KV recache of all 30 layers: K = RoPE(RMSNorm(X
+Wk)), V = X Wv for the 12 cached frames, X [18720, 1536]), then for each of
 the 40 latent frames and each of the 30 layers, RoPE + append of the frame's
-K/V into the layer's sink+ring cache, then sink-window attention of the
+K/V into the layer's sink+ring cache and sink-window attention of the
 frame's 1560 queries over the 12 cached frames (18720 keys). Inputs are
 seeded synthetic tensors, N(0,1)*0.5, from per-layer pools of 16 frames
 resident in HBM; the 30 caches (3.45 GB in bf16) exceed L2, so no L2 flush is
@@ -157,16 +159,48 @@ class Stream:
             self.k.append(W.normal(shape, base + 2, w.qkv_scale, torch.bfloat16, device))
             self.v.append(W.normal(shape, base + 3, w.qkv_scale, torch.bfloat16, device))
         self.out = torch.empty((1, w.N, w.H, w.D), dtype=torch.bfloat16, device=device)
+        # prompt-switch inputs per layer: hidden states of the 12 cached frames and the projections
+        dm = w.dm
+        self.rx, self.rwk, self.rwv, self.rg = [], [], [], []
+        for l in range(self.layers):
+            base = (w.seed * 7_919 + (l + seed_offset) * 104_729) & ((1 << 62) - 1)
+            self.rx.append(W.normal((1, w.slots * w.N, dm), base + 1, 1.0, torch.bfloat16, device))
+            self.rwk.append(W.normal((dm, w.H * w.D), base + 2, 1.0 / math.sqrt(dm), torch.bfloat16, device))
+            self.rwv.append(W.normal((dm, w.H * w.D), base + 3, 1.0 / math.sqrt(dm), torch.bfloat16, device))
+            self.rg.append(W.uniform((w.H * w.D,), base + 4, 0.5, 1.5, torch.float32, device))
         # fill every slot once so the segments below run in steady state
         for l in range(self.layers):
             for f in range(w.slots):
                 swa.kvcache_append(self.caches[l], self.k[l][f % POOL], self.v[l][f % POOL], f, self.rope)
         torch.cuda.synchronize()
 
-    def step(self, seg: int, attn_events=None, qkv=None):
-        """One 40-frame segment; frames 40*(seg+1) .. 40*(seg+1)+39."""
+    def held_frames(self, last: int):
+        """Frame held by each occupied cache slot once frames 0..last are
+        written (the library's slot map over the sinks and the last ring's
+        worth of frames)."""
+        w = self.w
+        held = [-1] * w.slots
+        for f in list(range(min(w.n_sink, last + 1))) + list(range(max(w.n_sink, last - w.n_local + 1), last + 1)):
+            held[self.swa.slot_of_frame(f, w.n_sink, w.n_local)] = f
+        return [f for f in held if f >= 0]
+
+    def step(self, seg: int, attn_events=None, qkv=None, recache_events=None):
+        """One 40-frame segment; frames 40*(seg+1) .. 40*(seg+1)+39, opened by a
+        prompt switch (recache of every layer)."""
         swa = self.swa
         launches = 0
+        first = SEGMENT * (seg + 1)
+        held = self.held_frames(first - 1)
+        if recache_events is not None:
+            recache_events[0].record()
+        for l in range(self.layers):
+            swa.kv_recache(self.caches[l], self.rx[l], self.rwk[l], self.rwv[l], self.rg[l], 1e-6, held, self.rope)
+            launches += 1
+        if recache_events is not None:
+            recache_events[1].record()
+            recache_events[2].append((recache_events[0], recache_events[1]))
+            recache_events[0] = torch.cuda.Event(enable_timing=True)
+            recache_events[1] = torch.cuda.Event(enable_timing=True)
         for i in range(SEGMENT):
             f = SEGMENT * (seg + 1) + i
             for l in range(self.layers):
@@ -211,13 +245,14 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0:
         clocks.start()
     ev = [torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True), []]
+    rev = [torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True), []]
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     barrier()
     t0.record()
     launches = 0
     for s in range(args.steps):
-        launches += st.step(args.warmup + s, attn_events=ev)
+        launches += st.step(args.warmup + s, attn_events=ev, recache_events=rev)
     t1.record()
     barrier()
     clk = clocks.stop() if rank == 0 else None
@@ -245,6 +280,9 @@ def run_ours(args, rank, world, local_rank):
     fl = attention_flops(w)
     achieved = fl / avg_attn_s / 1e12
     traffic = load_traffic()
+    recache_ms = [a.elapsed_time(b) for a, b in rev[2]]
+    rc_layer_s = (sum(recache_ms) / len(recache_ms)) / 1e3 / w.layers
+    rc_flops = 2.0 * (w.slots * w.N) * w.dm * (2 * w.H * w.D)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True,
@@ -253,13 +291,16 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": f"240s stream segment: {SEGMENT} latent frames x {w.layers} layers, H=12 D=128, "
                                f"1560 tok/frame, 3 sink + 9 local, LoL jitter 0.8, {args.cache} KV cache",
                    "frames_per_step": SEGMENT, "layers": w.layers, "tokens_per_frame": w.N, "keys": w.slots * w.N,
-                   "heads": w.H, "head_dim": w.D, "kv_cache": args.cache, "recache": "not in the step yet",
+                   "heads": w.H, "head_dim": w.D, "kv_cache": args.cache,
+                   "recache": f"all {w.layers} layers at the segment start (X [{w.slots * w.N}, {w.dm}])",
                    "l2": "inputs larger than L2 (30 caches x 115 MB)", "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "tensor", "kernel": "sink_window_attention_kernel",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_kind": f"{kind} bf16 dense, sustained",
                      "algorithmic_flops_per_launch": fl, "avg_launch_us": round(avg_attn_s * 1e6, 2)},
+        "recache_kernel": {"achieved_tflops": round(rc_flops / rc_layer_s / 1e12, 1),
+                           "us_per_layer": round(rc_layer_s * 1e6, 2), "flops_per_layer": rc_flops},
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clk,
@@ -283,7 +324,9 @@ def run_e2e(st: Stream, args, barrier, dist):
     free = [torch.cuda.Event() for _ in range(2)]
     for e in free:
         e.record(comp)
-    h2d = 3 * w.N * w.H * w.D * 2 * L * SEGMENT
+    host_x = st.rx[0].cpu().pin_memory()      # the prompt-switch hidden states of one layer
+    x_ready = torch.cuda.Event()
+    h2d = 3 * w.N * w.H * w.D * 2 * L * SEGMENT + host_x.numel() * 2 * L
     d2h = w.N * w.H * w.D * 2 * SEGMENT
 
     def seg(s, start=None):
@@ -298,6 +341,17 @@ def run_e2e(st: Stream, args, barrier, dist):
                         t_dev.copy_(t_host, non_blocking=True)
                 ready[b].record(copy)
 
+        held = st.held_frames(SEGMENT * (s + 1) - 1)
+        with torch.cuda.stream(copy):             # every layer's X crosses PCIe at the switch
+            if start is not None:
+                copy.wait_event(start)
+            copy.wait_stream(comp)
+            for l in range(L):
+                st.rx[l].copy_(host_x, non_blocking=True)
+            x_ready.record(copy)
+        comp.wait_event(x_ready)
+        for l in range(L):
+            st.swa.kv_recache(st.caches[l], st.rx[l], st.rwk[l], st.rwv[l], st.rg[l], 1e-6, held, st.rope)
         load(0)
         for i in range(SEGMENT):
             if i + 1 < SEGMENT:
@@ -484,6 +538,33 @@ def run_attention_only(args):
             "frac_of_burst_peak": round(fl / t / 1e12 / peaks["bf16_tflops"], 4), "peak_kind": kind}
 
 
+def run_recache_only(args):
+    """One layer's KV recache at the Wan shape (X [18720, 1536], Wk, Wv
+    [1536, 1536]): `warmup` + `steps` launches timed with CUDA events."""
+    from sink_window_attention_b200 import build
+    build.build()
+    import sink_window_attention_b200 as swa
+    st = Stream(W.replace(W.STREAM, layers=1), "bf16", "cuda")
+    held = st.held_frames(SEGMENT - 1)
+    times = []
+    for i in range(args.warmup + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        swa.kv_recache(st.caches[0], st.rx[0], st.rwk[0], st.rwv[0], st.rg[0], 1e-6, held, st.rope)
+        b.record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(a.elapsed_time(b) / 1e3)
+    assert swa.device_error() == 0
+    w = st.w
+    fl = 2.0 * (w.slots * w.N) * w.dm * (2 * w.H * w.D)
+    peaks, kind = measured_peaks()
+    t = statistics.median(times)
+    return {"mode": "recache", "launches": len(times), "median_us": round(t * 1e6, 2),
+            "tflops": round(fl / t / 1e12, 1), "frac_of_burst_peak": round(fl / t / 1e12 / peaks["bf16_tflops"], 4),
+            "peak_kind": kind}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -494,11 +575,14 @@ def main():
     ap.add_argument("--layers", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
-    ap.add_argument("--mode", default="stream", choices=["stream", "attention"])
+    ap.add_argument("--mode", default="stream", choices=["stream", "attention", "recache"])
     ap.add_argument("--workload", default="wan", choices=["wan", "chunk"])
     args = ap.parse_args()
     if args.mode == "attention":
         print(json.dumps(run_attention_only(args)), flush=True)
+        return
+    if args.mode == "recache":
+        print(json.dumps(run_recache_only(args)), flush=True)
         return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

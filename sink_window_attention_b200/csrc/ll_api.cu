@@ -11,6 +11,7 @@
 #include "../../include/ll_api.h"
 #include "ll_attention.cuh"
 #include "ll_common.cuh"
+#include "ll_recache.cuh"
 #include "ll_rope_append.cuh"
 
 namespace {
@@ -410,16 +411,100 @@ size_t ll_kv_recache_workspace_bytes(const ll_kvcache* cache, int d_model, int n
   (void)cache;
   (void)d_model;
   (void)n_slots;
-  return 0;
+  return 0;  // the recache kernel needs no scratch
 }
 
 ll_status ll_kv_recache(const ll_kvcache* cache, const void* x, int d_model, const void* wk, const void* wv,
                         const float* gamma, float rms_eps, const long long* slot_frames, int n_slots,
                         const ll_rope_desc* rope, void* workspace, size_t workspace_bytes, void* stream) {
   g_last_error.clear();
-  (void)cache; (void)x; (void)d_model; (void)wk; (void)wv; (void)gamma; (void)rms_eps;
-  (void)slot_frames; (void)n_slots; (void)rope; (void)workspace; (void)workspace_bytes; (void)stream;
-  return fail(LL_ERR_UNSUPPORTED, "kv recache is not built yet");
+  (void)workspace;
+  (void)workspace_bytes;
+  ll_status st = check_cache(cache);
+  if (st != LL_OK) return st;
+  if (x == nullptr || wk == nullptr || wv == nullptr || gamma == nullptr || slot_frames == nullptr)
+    return fail(LL_ERR_INVALID_ARG, "x, wk, wv, gamma and slot_frames must be non-NULL");
+  if (!aligned16(x) || !aligned16(wk) || !aligned16(wv))
+    return fail(LL_ERR_INVALID_ARG, "x, wk and wv must be 16-byte aligned");
+  const int S = cache->n_sink + cache->n_local;
+  if (n_slots < 1 || n_slots > S || n_slots > ll::kMaxSlots)
+    return fail(LL_ERR_INVALID_ARG, "n_slots = %d must lie in [1, %d]", n_slots, S < ll::kMaxSlots ? S : ll::kMaxSlots);
+  for (int i = 0; i < n_slots; ++i)
+    if (slot_frames[i] < 0) return fail(LL_ERR_INVALID_ARG, "slot_frames[%d] is negative", i);
+  if (!(rms_eps >= 0.f) || !std::isfinite(rms_eps)) return fail(LL_ERR_INVALID_ARG, "rms_eps must be finite, >= 0");
+  if ((st = check_grid(rope, cache->tokens_per_frame)) != LL_OK) return st;
+  if (cache->dtype != LL_BF16 && cache->dtype != LL_FP8_E4M3)
+    return fail(LL_ERR_UNSUPPORTED, "kv recache writes BF16 or FP8 caches");
+  const int Dout = cache->H * cache->D;
+  if (d_model < 64 || d_model % 64 != 0)
+    return fail(LL_ERR_UNSUPPORTED, "d_model = %d must be a positive multiple of 64", d_model);
+  if (Dout % 256 != 0 || Dout / 256 > 8 || (cache->D != 64 && cache->D != 128))
+    return fail(LL_ERR_UNSUPPORTED, "H*D = %d must be a multiple of 256 up to 2048 with D = 64 or 128", Dout);
+  using TR = ll::RecacheTraits;
+  ll::RecacheParams p{};
+  if ((st = make_rope(rope, cache->H, cache->D, 0, &p.rp)) != LL_OK) return st;
+  p.k_cache = cache->k;
+  p.v_cache = cache->v;
+  p.k_scale = cache->k_scale;
+  p.v_scale = cache->v_scale;
+  p.gamma = gamma;
+  p.eps = rms_eps;
+  p.M = n_slots * cache->tokens_per_frame;
+  p.Din = d_model;
+  p.Dout = Dout;
+  p.H = cache->H;
+  p.D = cache->D;
+  p.N = cache->tokens_per_frame;
+  p.S = S;
+  p.fp8 = cache->dtype == LL_FP8_E4M3;
+  for (int i = 0; i < n_slots; ++i) p.slot_frame[i] = static_cast<int>(slot_frames[i]);
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(LL_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  CUtensorMap tmX, tmWk, tmWv;
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)d_model, (cuuint64_t)p.M, (cuuint64_t)cache->B};
+    const cuuint64_t strides[2] = {(cuuint64_t)d_model * 2, (cuuint64_t)p.M * d_model * 2};
+    const cuuint32_t box[3] = {64u, 128u, 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    if (fn(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(x), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return fail(LL_ERR_CUDA, "cuTensorMapEncodeTiled(x) failed");
+  }
+  for (int w = 0; w < 2; ++w) {
+    const cuuint64_t dims[2] = {(cuuint64_t)Dout, (cuuint64_t)d_model};
+    const cuuint64_t strides[1] = {(cuuint64_t)Dout * 2};
+    const cuuint32_t box[2] = {64u, 64u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    if (fn(w ? &tmWv : &tmWk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w ? wv : wk), dims, strides,
+           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return fail(LL_ERR_CUDA, "cuTensorMapEncodeTiled(w) failed");
+  }
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(ll::kv_recache_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TR::SMEM_BYTES) !=
+        cudaSuccess)
+      return check_launch("cudaFuncSetAttribute(recache)");
+    if (cudaFuncSetAttribute(ll::kv_recache_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess)
+      return check_launch("cudaFuncSetAttribute(recache cluster)");
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(Dout / TR::BN, (p.M + TR::BM - 1) / TR::BM, 2 * cache->B);
+  cfg.blockDim = dim3(TR::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = TR::SMEM_BYTES;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = Dout / TR::BN;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, ll::kv_recache_kernel, tmX, tmWk, tmWv, p) != cudaSuccess)
+    return check_launch("kv_recache_kernel");
+  return check_launch("kv_recache_kernel");
 }
 
 }  // extern "C"

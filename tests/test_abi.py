@@ -113,3 +113,18 @@ def test_append_and_rope_validation(L):
     assert L.ll_rope_apply(None, swa.LL_BF16, 1, 1, 12, 128, 0, rc, None) == swa.LL_ERR_INVALID_ARG
     assert L.ll_rope_apply(k, swa.LL_FP8_E4M3, 1, 1, 12, 128, 0, rc, None) == swa.LL_ERR_INVALID_ARG
     assert L.ll_rope_apply(k, swa.LL_BF16, 1, 1, 12, 128, 0, None, None) == swa.LL_ERR_INVALID_ARG
+
+
+def test_recache_validation(L):
+    c = _cache()
+    frames = (ctypes.c_longlong * 12)(*range(12))
+    g = 1 << 22
+    def call(cache=c, n=12, dm=1536, fr=frames, x=1 << 20):
+        return L.ll_kv_recache(ctypes.byref(cache), x, dm, 1 << 21, 1 << 21, g, 1e-6, fr, n, None, None, 0, None)
+    assert call(n=0) == swa.LL_ERR_INVALID_ARG
+    assert call(n=13) == swa.LL_ERR_INVALID_ARG
+    assert call(x=None) == swa.LL_ERR_INVALID_ARG
+    assert call(fr=(ctypes.c_longlong * 12)(*([-1] * 12))) == swa.LL_ERR_INVALID_ARG
+    assert call(dm=100) == swa.LL_ERR_UNSUPPORTED
+    assert call(cache=_cache(H=3)) == swa.LL_ERR_UNSUPPORTED        # H*D = 384 is not a multiple of 256
+    assert call(cache=_cache(dtype=swa.LL_F32)) == swa.LL_ERR_UNSUPPORTED
