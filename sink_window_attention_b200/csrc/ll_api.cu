@@ -191,6 +191,21 @@ ll_status launch_attention(ll::AttnParams p, const ll_kvcache* c, long long S, v
   return check_launch("sink_window_attention_kernel");
 }
 
+// Bytes of the bf16 copy of an FP8 cache that attention over an FP8 cache
+// dequantises into (placed after the attention scratch in the workspace).
+size_t fp8_staging_half(const ll_kvcache* c) {  // one of K / V, bf16, 256-byte aligned
+  const size_t S = static_cast<size_t>(c->n_sink + c->n_local);
+  return align256(static_cast<size_t>(c->B) * S * c->tokens_per_frame * c->H * c->D * sizeof(__nv_bfloat16));
+}
+size_t fp8_staging_bytes(const ll_kvcache* c) { return c->dtype == LL_FP8_E4M3 ? 2 * fp8_staging_half(c) : 0; }
+
+size_t attention_scratch_bytes(const ll_kvcache* cache, int n_query_frames) {
+  const int units = ((n_query_frames * cache->tokens_per_frame + 127) / 128) * cache->H * cache->B;
+  if (cache->D == 128) return align256(attention_workspace<ll::AttnTraits<128, __nv_bfloat16>>(units));
+  if (cache->dtype == LL_F32) return align256(attention_workspace<ll::AttnTraits<64, float>>(units));
+  return align256(attention_workspace<ll::AttnTraits<64, __nv_bfloat16>>(units));
+}
+
 }  // namespace
 
 extern "C" {
@@ -303,10 +318,7 @@ ll_status ll_kvcache_append(const ll_kvcache* cache, const void* k, const void* 
 size_t ll_sink_window_attention_workspace_bytes(const ll_kvcache* cache, int n_query_frames) {
   if (cache == nullptr || n_query_frames < 1 || cache->tokens_per_frame < 1 || cache->H < 1 || cache->B < 1)
     return 0;
-  const int units = ((n_query_frames * cache->tokens_per_frame + 127) / 128) * cache->H * cache->B;
-  if (cache->D == 128) return attention_workspace<ll::AttnTraits<128, __nv_bfloat16>>(units);
-  if (cache->dtype == LL_F32) return attention_workspace<ll::AttnTraits<64, float>>(units);
-  return attention_workspace<ll::AttnTraits<64, __nv_bfloat16>>(units);
+  return attention_scratch_bytes(cache, n_query_frames) + fp8_staging_bytes(cache);
 }
 
 ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvcache* cache, long long first_frame,
@@ -331,10 +343,42 @@ ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvc
   const bool f32 = cache->dtype == LL_F32;
   if (f32 ? q_dtype != LL_F32 : q_dtype != LL_BF16)
     return fail(LL_ERR_INVALID_ARG, "q dtype must be F32 for an F32 cache and BF16 otherwise");
-  if (cache->dtype == LL_FP8_E4M3) return fail(LL_ERR_UNSUPPORTED, "attention over an FP8 cache is not built yet");
   const long long S = cache->n_sink + cache->n_local;
   const long long last = first_frame + n_query_frames - 1;
   const long long valid_slots = last + 1 < S ? last + 1 : S;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ll_kvcache staged;
+  if (cache->dtype == LL_FP8_E4M3) {
+    // E4M3 cache: the occupied rows are dequantised into bf16 staging inside
+    // the workspace, then the bf16 kernel runs on the staged copy
+    if (cache->D != 128 && cache->D != 64)
+      return fail(LL_ERR_UNSUPPORTED, "attention supports D = 64 or 128; got D = %d", cache->D);
+    const size_t half = fp8_staging_half(cache);
+    char* stage = static_cast<char*>(workspace) + attention_scratch_bytes(cache, n_query_frames);
+    ll::DequantParams dp{};
+    dp.src[0] = static_cast<const uint8_t*>(cache->k);
+    dp.src[1] = static_cast<const uint8_t*>(cache->v);
+    dp.scale[0] = cache->k_scale;
+    dp.scale[1] = cache->v_scale;
+    dp.dst[0] = reinterpret_cast<__nv_bfloat16*>(stage);
+    dp.dst[1] = reinterpret_cast<__nv_bfloat16*>(stage + half);
+    dp.B = cache->B;
+    dp.rows = static_cast<int>(valid_slots * cache->tokens_per_frame);
+    dp.batch_rows = static_cast<int>(S * cache->tokens_per_frame);
+    dp.H = cache->H;
+    dp.D = cache->D;
+    const long long chunks = static_cast<long long>(dp.B) * dp.rows * dp.H * (dp.D / 16);
+    const long long want = (chunks + 255) / 256;
+    const dim3 grid(static_cast<unsigned>(want < 8LL * num_sms() ? want : 8LL * num_sms()), 2);
+    ll::dequant_e4m3_kernel<<<grid, 256, 0, s>>>(dp);
+    if ((st = check_launch("dequant_e4m3_kernel")) != LL_OK) return st;
+    staged = *cache;
+    staged.k = dp.dst[0];
+    staged.v = dp.dst[1];
+    staged.k_scale = staged.v_scale = nullptr;
+    staged.dtype = LL_BF16;
+    cache = &staged;
+  }
   ll::AttnParams p{};
   if ((st = make_rope(rope, cache->H, cache->D, first_frame, &p.rp)) != LL_OK) return st;
   p.q = q;
@@ -346,7 +390,6 @@ ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvc
   p.Nk = static_cast<int>(valid_slots * cache->tokens_per_frame);
   p.softmax_scale = softmax_scale;
   p.N = cache->tokens_per_frame;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!f32 && cache->D == 128)
     return launch_attention<ll::AttnTraits<128, __nv_bfloat16>>(p, cache, S, workspace, workspace_bytes, s);
   if (!f32 && cache->D == 64)

@@ -8,6 +8,7 @@
 #pragma once
 
 #include "ll_common.cuh"
+#include <cuda_fp16.h>
 
 namespace ll {
 
@@ -262,6 +263,48 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
         store_chunk8<C>(static_cast<C*>(p.v_cache) + drow * p.D + c * 8, vx);
       }
     }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// E4M3 cache rows -> bf16: value = decode(code) * scale for the first `rows`
+// token rows of every batch entry, K and V (blockIdx.y = 0 / 1). 16 codes
+// (16 bytes) per thread.
+// ---------------------------------------------------------------------------
+struct DequantParams {
+  const uint8_t* src[2];
+  const float* scale[2];
+  __nv_bfloat16* dst[2];
+  int B, rows, batch_rows, H, D;
+};
+
+__global__ void __launch_bounds__(256) dequant_e4m3_kernel(const DequantParams p) {
+  const int which = blockIdx.y;
+  const int cpr = p.D / 16;  // 16-code chunks per (token, head) row
+  const int per_batch = p.rows * p.H * cpr;
+  const int total = p.B * per_batch;
+  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += gridDim.x * blockDim.x) {
+    const int b = idx / per_batch;
+    const int r = idx - b * per_batch;         // (token * H + h) * cpr + c within the batch entry
+    const int th = r / cpr, c = r - th * cpr;  // token-head row, chunk
+    const size_t row = static_cast<size_t>(b) * p.batch_rows * p.H + th;
+    const float sc = p.scale[which][row];
+    const uint4 u = *reinterpret_cast<const uint4*>(p.src[which] + row * p.D + c * 16);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const __nv_fp8x2_storage_t q = static_cast<__nv_fp8x2_storage_t>((w[i] >> (16 * half)) & 0xFFFFu);
+        const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(q, __NV_E4M3);
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+        o[2 * i + half] = pack_bf16(f.x * sc, f.y * sc);
+      }
+    }
+    uint4* d = reinterpret_cast<uint4*>(p.dst[which] + row * p.D + c * 16);
+    d[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    d[1] = make_uint4(o[4], o[5], o[6], o[7]);
   }
 }
 
