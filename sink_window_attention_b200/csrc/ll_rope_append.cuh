@@ -80,6 +80,32 @@ __device__ __forceinline__ void rotate_chunk8(float (&x)[8], int j0, float pos_t
   }
 }
 
+// sin and cos of x for |x| up to ~1e5: Cody and Waite's two-constant
+// reduction x = k 2pi + r (k = rint(x / 2pi); 2pi split into its float
+// rounding and the remainder, each product taken in one FMA) brings r into
+// [-pi, pi], where the hardware approximation is accurate to ~4e-7 absolute.
+__device__ __forceinline__ void sincos_reduced(float x, float& s, float& c) {
+  const float k = rintf(x * 0.15915494309189535f);
+  float r = fmaf(-k, 6.28318548202514648f, x);
+  r = fmaf(k, 1.7484555314695172e-7f, r);
+  __sincosf(r, &s, &c);
+}
+
+// rotate_chunk8 with sincos_reduced (query tiles staged by the attention kernel)
+__device__ __forceinline__ void rotate_chunk8_fast(float (&x)[8], int j0, float pos_t, float pos_r, float pos_c,
+                                                   const float* omega_h, int pt, int pth) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int j = j0 + q;
+    const float pos = j < pt ? pos_t : (j < pth ? pos_r : pos_c);
+    float s, c;
+    sincos_reduced(pos * omega_h[j], s, c);
+    const float a = x[2 * q], b = x[2 * q + 1];
+    x[2 * q] = a * c - b * s;
+    x[2 * q + 1] = a * s + b * c;
+  }
+}
+
 template <typename T>
 __device__ __forceinline__ void load_chunk8(const T* p, float (&x)[8]);
 template <>
