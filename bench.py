@@ -135,6 +135,29 @@ def gpu_index_for(local_rank: int) -> str:
     return str(local_rank)
 
 
+def replica_seed_offset(rank: int) -> int:
+    """Replicas stream different synthetic inputs: rank r offsets every layer
+    seed by 1000 r (30 layers per rank, so no two ranks share a seed)."""
+    return 1000 * rank
+
+
+def layer_seed_base(w: W.Workload, layer: int, seed_offset: int) -> int:
+    """Seed of one layer's Q/K/V input pools (the pools use base + 1, 2, 3)."""
+    return (w.seed * 1_000_003 + (layer + seed_offset) * 10_007) & ((1 << 62) - 1)
+
+
+def max_over_ranks(value: float, dist: bool, device: str = "cuda") -> float:
+    """The slowest rank's device time. Every rank calls it at the same point
+    (one collective, same order on all ranks); without a process group it is
+    the identity."""
+    if not dist:
+        return value
+    import torch.distributed as tdist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
@@ -154,7 +177,7 @@ class Stream:
         shape = (POOL, 1, w.N, w.H, w.D)
         self.q, self.k, self.v = [], [], []
         for l in range(self.layers):
-            base = (w.seed * 1_000_003 + (l + seed_offset) * 10_007) & ((1 << 62) - 1)
+            base = layer_seed_base(w, l, seed_offset)
             self.q.append(W.normal(shape, base + 1, w.qkv_scale, torch.bfloat16, device))
             self.k.append(W.normal(shape, base + 2, w.qkv_scale, torch.bfloat16, device))
             self.v.append(W.normal(shape, base + 3, w.qkv_scale, torch.bfloat16, device))
@@ -230,7 +253,7 @@ def run_ours(args, rank, world, local_rank):
     import sink_window_attention_b200 as swa
     w = W.STREAM if args.cache == "bf16" else W.STREAM_FP8
     w = W.replace(w, layers=args.layers)
-    st = Stream(w, "bf16" if args.cache == "bf16" else "fp8", "cuda", seed_offset=1000 * rank)
+    st = Stream(w, "bf16" if args.cache == "bf16" else "fp8", "cuda", seed_offset=replica_seed_offset(rank))
     dist = world > 1
     if dist:
         import torch.distributed as tdist
@@ -263,10 +286,7 @@ def run_ours(args, rank, world, local_rank):
     dev_err = swa.device_error()
     if dev_err:
         raise RuntimeError(f"device error word {dev_err}")
-    if dist:
-        t = torch.tensor([ms], device="cuda")
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist)
 
     # ---- end to end through the public API with host buffers (pinned), per step:
     # every frame's Q/K/V of every layer is copied host -> device on a copy
@@ -379,12 +399,7 @@ def run_e2e(st: Stream, args, barrier, dist):
         seg(args.warmup + args.steps + 1 + s, start=a if s == 0 else None)
     bb.record()
     barrier()
-    ms = a.elapsed_time(bb)
-    if dist:
-        import torch.distributed as tdist
-        t = torch.tensor([ms], device="cuda")
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(a.elapsed_time(bb), dist)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     return {"value": round(SEGMENT * steps * world / (ms / 1e3), 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": steps}
