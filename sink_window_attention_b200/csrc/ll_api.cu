@@ -173,7 +173,10 @@ ll_status launch_attention(ll::AttnParams p, const ll_kvcache* c, long long S, v
   CUtensorMap tmK, tmV;
   const CUtensorMapDataType dt = TR::ES == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   const long long batch_rows = S * c->tokens_per_frame;
-  ll_status st = encode_rows_map(&tmK, c->k, dt, TR::ES, TR::D, c->H, p.Nk, batch_rows, c->B, TR::BN);
+  CUtensorMap tmQ;
+  ll_status st = encode_rows_map(&tmQ, p.q, dt, TR::ES, TR::D, c->H, p.Tq, p.Tq, c->B, TR::BM);
+  if (st != LL_OK) return st;
+  st = encode_rows_map(&tmK, c->k, dt, TR::ES, TR::D, c->H, p.Nk, batch_rows, c->B, TR::BN);
   if (st != LL_OK) return st;
   st = encode_rows_map(&tmV, c->v, dt, TR::ES, TR::D, c->H, p.Nk, batch_rows, c->B, TR::BN,
                        TR::ES == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B);
@@ -187,7 +190,7 @@ ll_status launch_attention(ll::AttnParams p, const ll_kvcache* c, long long S, v
   }
   if (cudaMemsetAsync(p.counters, 0, p.units * sizeof(int), stream) != cudaSuccess)
     return check_launch("cudaMemsetAsync(attention counters)");
-  kern<<<p.grid, TR::THREADS, TR::SMEM_BYTES, stream>>>(tmK, tmV, p);
+  kern<<<p.grid, TR::THREADS, TR::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
   return check_launch("sink_window_attention_kernel");
 }
 

@@ -18,24 +18,20 @@
 //    [B][S*N][H][D] cache with 4D TMA loads (128-byte swizzle; rows past the
 //    valid keys read as zeros). K and V have rings and cursors of their own,
 //    each refilled as soon as a stage frees, so K runs ahead of V.
-//  * warps 2-3 load the next piece's Q tile with 128-bit loads, apply the 3D
-//    RoPE in registers (angles reduced to [-pi, pi], then the hardware
-//    sine/cosine) and write the swizzled operand layout into the free half of
-//    a double-buffered Q, so RoPE costs no extra pass over Q.
-//  * warp 1 owns 512 TMEM columns: S_A, S_B, one O accumulator and P_A, P_B.
-//    One lane issues tcgen05.mma whenever an operand is ready: S_i = Q K_i^T
-//    into S_(i mod 2) as soon as the softmax has read the previous S from it
-//    (P lives in its own columns, so S is free early), and O += P_i V_i (the
-//    A operand read from tensor memory).
-//  * two softmax warpgroups take the key tiles of a piece in turn (warps 4-7:
-//    even tiles, warps 8-11: odd ones; one query row per thread, one TMEM lane
-//    quarter per warp). They share one running max, handed from tile to tile
-//    through shared memory; O is rescaled in TMEM by the warpgroup whose tile
-//    raised the max by more than 2^8 (after the previous P V completed, before
-//    its own), so with lazy rescaling both warpgroups work almost
-//    independently while the tensor core keeps one O. Each warpgroup keeps
-//    its own row sums relative to the max it last used; the two are combined
-//    at the end of a piece.
+//  * Q tiles come in by TMA (the same swizzled operand layout, rows past the
+//    query count zero-filled) into a double buffer; warps 2-3 then apply the
+//    3D RoPE in place in shared memory (angles reduced to [-pi, pi], then the
+//    hardware sine/cosine), so RoPE costs no extra pass over Q in HBM.
+//  * warp 1 owns 512 TMEM columns: S_A, S_B (128 each) and O_A, O_B. One lane
+//    issues tcgen05.mma: S_i = Q K_i^T into S_(i mod 2) and O_(i mod 2) +=
+//    P_i V_i, where P_i sits in the TMEM columns of S_i (the A operand is read
+//    from tensor memory), so P never touches shared memory.
+//  * two softmax warpgroups (warps 4-7: even key tiles of a piece, warps 8-11:
+//    odd ones; one query row per thread, one TMEM lane quarter per warp) keep
+//    independent running (max, sum) and O; O is rescaled in TMEM only when the
+//    running max grows by more than 2^8 (the final division uses the same max,
+//    so the result is unchanged). At the end of a piece warpgroup A merges
+//    the two halves.
 //  * Every mbarrier wait is bounded; a wait that gives up records an error,
 //    raises an abort flag the other roles see, and all roles still walk the
 //    same named-barrier sequence so nothing can hang. TMEM accesses
@@ -65,22 +61,14 @@ struct AttnTraits {
   static constexpr int FMT = (ES == 2) ? 1 : 2;     // bf16 / tf32
   static constexpr int QST = 2;                     // Q buffers
   static constexpr int EXP_FMA_FROM = 8;            // pairs e with (e % 8) >= this use exp2_fma_x2 (8: none)
-  static constexpr int CTRL_BYTES = 3072;
-  static constexpr int STAGE_BUDGET = 232448 - CTRL_BYTES - QST * Q_BYTES;
+  static constexpr int CTRL_BYTES = 2048;
+  static constexpr int STAGE_BUDGET = 232448 - CTRL_BYTES - 1024 - QST * Q_BYTES;
   static constexpr int STAGES = STAGE_BUDGET / KV_BYTES;
   static constexpr int KST = STAGES >= 8 ? 4 : (STAGES + 1) / 2;
   static constexpr int VST = STAGES >= 8 ? 4 : STAGES - KST;
-  // the dynamic shared memory base is 1024-byte aligned (checked on entry)
-  static constexpr int SMEM_BYTES = CTRL_BYTES + QST * Q_BYTES + (KST + VST) * KV_BYTES;
-  // TMEM: S_A, S_B (BN fp32 columns each), one O (D columns) and, for bf16,
-  // separate P_A, P_B (BN/2 columns of packed bf16 pairs); tf32 keeps P in
-  // the columns of its S (one fp32 per column would not fit).
+  static constexpr int SMEM_BYTES = CTRL_BYTES + 1024 + QST * Q_BYTES + (KST + VST) * KV_BYTES;
   static constexpr int TMEM_COLS = 512;
-  static constexpr bool P_SEPARATE = (ES == 2);
-  static constexpr int P_COLS = BN * ES / 4;
-  static constexpr int O_COL = 2 * BN;
-  static constexpr int P_COL0 = P_SEPARATE ? O_COL + D : 0;  // P_w at P_COL0 + w * (P_SEPARATE ? P_COLS : BN)
-  static constexpr int P_STRIDE = P_SEPARATE ? P_COLS : BN;
+  static constexpr int S_COL0 = 0, O_COL0 = 2 * BN;  // S_w at w*BN, O_w at O_COL0 + w*D
   static constexpr int THREADS = 384;
   // register split: launch 168 per thread (384 x 168 = 64512); warpgroup 0
   // (producer, MMA, Q loader) gives up 96 per thread, the two softmax
@@ -88,11 +76,10 @@ struct AttnTraits {
   // that ptxas allocated exactly LAUNCH_REGS.
   static constexpr int LAUNCH_REGS = 168, REGS_LOW = 72, REGS_HIGH = 216;
   static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= THREADS * LAUNCH_REGS, "register split exceeds the launch");
-  static_assert(REGS_LOW % 8 == 0 && REGS_HIGH % 8 == 0, "setmaxnreg takes multiples of 8");
   static constexpr int SLOT_FLOATS = BM * D + 2 * BM;  // one partial: O rows, then m, then l
   static_assert(KST >= 2 && VST >= 2, "need at least two K and two V stages");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-  static_assert(O_COL + D + (P_SEPARATE ? 2 * P_COLS : 0) <= TMEM_COLS, "TMEM budget");
+  static_assert(O_COL0 + 2 * D <= TMEM_COLS, "TMEM budget");
   static_assert(NB >= 1 && ROWB % 128 == 0, "rows must be whole 128-byte blocks");
 };
 
@@ -126,77 +113,73 @@ __device__ __forceinline__ int owner_of(long long i, long long total, int G) {
 
 // Q tile of unit u, rotated with this head's frequencies `om` [D/2], into
 // the 128-byte-swizzled K-major operand layout at sQ.
-template <class TR, int BATCH>
-__device__ __forceinline__ void load_q_tile(uint8_t* sQ, const AttnParams& p, const float* om, int u, int tid,
-                                            int nthreads) {
+// Apply the 3D RoPE in place to a Q tile that TMA has put into shared memory
+// (128-byte swizzled, K-major: the operand layout the MMA reads). Rows past
+// Tq were zero-filled by TMA and stay zero. Each thread takes 8-element
+// groups; rotation in fp32, rounded back to the tile's type.
+template <class TR>
+__device__ __forceinline__ void rope_q_tile_inplace(uint8_t* sQ, const AttnParams& p, const float* om, int u, int tid,
+                                                    int nthreads) {
   using T = typename TR::T;
   constexpr int BM = TR::BM, D = TR::D;
-  const int qt = u % p.q_tiles;
-  const int h = (u / p.q_tiles) % p.H;
-  const int b = u / (p.q_tiles * p.H);
-  const int q0 = qt * BM;
-  const T* q = static_cast<const T*>(p.q);
   constexpr int GPR = D / 8;  // 8-element groups per row
-  // BATCH global loads in flight per thread
+  const int q0 = (u % p.q_tiles) * BM;
   const int pth = p.rp.pt + p.rp.ph;
-  for (int g0 = tid; g0 < BM * GPR; g0 += BATCH * nthreads) {
-    float x[BATCH][8];
+  for (int g = tid; g < BM * GPR; g += nthreads) {
+    const int r = g / GPR, e8 = g - r * GPR;
+    const int t = q0 + r;
+    if (t >= p.Tq) continue;
+    const int fi = t / p.N, n = t - fi * p.N;
+    const int rr = n / p.rp.grid_w, cc = n - rr * p.rp.grid_w;
+    float x[8];
+    if constexpr (TR::ES == 2) {
+      uint4* ptr = reinterpret_cast<uint4*>(sQ + (e8 >> 3) * (BM * 128) + sw128_offset(r, e8 & 7));
+      const uint4 v = *ptr;
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int k = 0; k < BATCH; ++k) {
-      const int g = g0 + k * nthreads;
-      const int r = g / GPR, e8 = g - r * GPR;
-      const int t = q0 + r;
-      if (g < BM * GPR && t < p.Tq) {
-        load_chunk8<T>(q + ((static_cast<size_t>(b) * p.Tq + t) * p.H + h) * D + e8 * 8, x[k]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x[k][i] = 0.f;
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
       }
-    }
-#pragma unroll
-    for (int k = 0; k < BATCH; ++k) {
-      const int g = g0 + k * nthreads;
-      if (g >= BM * GPR) break;
-      const int r = g / GPR, e8 = g - r * GPR;
-      const int t = q0 + r;
-      if (p.rp.enabled && t < p.Tq) {
-        const int fi = t / p.N, n = t - fi * p.N;
-        const int rr = n / p.rp.grid_w, cc = n - rr * p.rp.grid_w;
-        rotate_chunk8_fast(x[k], e8 * 4, static_cast<float>(p.rp.t_first + fi), static_cast<float>(rr),
-                      static_cast<float>(cc), om, p.rp.pt, pth);
-      }
-      if constexpr (TR::ES == 2) {
-        const int chunk = e8;  // 8 bf16 = 16 bytes
-        uint4 v;
-        v.x = pack_bf16(x[k][0], x[k][1]);
-        v.y = pack_bf16(x[k][2], x[k][3]);
-        v.z = pack_bf16(x[k][4], x[k][5]);
-        v.w = pack_bf16(x[k][6], x[k][7]);
-        *reinterpret_cast<uint4*>(sQ + (chunk >> 3) * (BM * 128) + sw128_offset(r, chunk & 7)) = v;
-      } else {
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int chunk = e8 * 2 + hh;  // 4 floats = 16 bytes
-          *reinterpret_cast<float4*>(sQ + (chunk >> 3) * (BM * 128) + sw128_offset(r, chunk & 7)) =
-              make_float4(x[k][4 * hh], x[k][4 * hh + 1], x[k][4 * hh + 2], x[k][4 * hh + 3]);
-        }
-      }
+      rotate_chunk8_fast(x, e8 * 4, static_cast<float>(p.rp.t_first + fi), static_cast<float>(rr),
+                         static_cast<float>(cc), om, p.rp.pt, pth);
+      *ptr = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
+    } else {
+      float4* p0 = reinterpret_cast<float4*>(sQ + ((2 * e8) >> 3) * (BM * 128) + sw128_offset(r, (2 * e8) & 7));
+      float4* p1 = reinterpret_cast<float4*>(sQ + ((2 * e8 + 1) >> 3) * (BM * 128) + sw128_offset(r, (2 * e8 + 1) & 7));
+      const float4 a = *p0, b = *p1;
+      x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+      x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+      rotate_chunk8_fast(x, e8 * 4, static_cast<float>(p.rp.t_first + fi), static_cast<float>(rr),
+                         static_cast<float>(cc), om, p.rp.pt, pth);
+      *p0 = make_float4(x[0], x[1], x[2], x[3]);
+      *p1 = make_float4(x[4], x[5], x[6], x[7]);
     }
   }
-  fence_proxy_async_smem();
+  fence_proxy_async_smem();  // the generic-proxy writes are read by the tensor core
+}
+
+// TMA copy of the Q tile of unit u into a Q buffer (NB column blocks of 128
+// bytes x BM rows; rows past Tq read as zeros). One thread.
+template <class TR>
+__device__ __forceinline__ void tma_q_tile(uint8_t* dst, const CUtensorMap* tmQ, uint64_t* bar, const AttnParams& p,
+                                           int u) {
+  const int qt = u % p.q_tiles, h = (u / p.q_tiles) % p.H, b = u / (p.q_tiles * p.H);
+  mbar_expect_tx(bar, TR::Q_BYTES);
+#pragma unroll
+  for (int blk = 0; blk < TR::NB; ++blk)
+    tma_load_4d(dst + blk * (TR::BM * 128), tmQ, bar, blk * TR::ELEMS_PER_BLOCK, h, qt * TR::BM, b);
 }
 
 template <class TR>
 __global__ void __launch_bounds__(384, 1)
-    sink_window_attention_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                                 const AttnParams p) {
+    sink_window_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                                 const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
   using T = typename TR::T;
   constexpr int BM = TR::BM, BN = TR::BN, D = TR::D, KST = TR::KST, VST = TR::VST;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  if ((smem_addr(smem) & 1023u) != 0) {  // the swizzled layouts need 1024-byte aligned buffers
-    if (threadIdx.x == 0) atomicOr(&g_error_word, kErrWaitTimeout);
-    return;
-  }
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                              // [QST][Q_BYTES]
   uint8_t* sK = sQ + TR::QST * TR::Q_BYTES;        // [KST][KV_BYTES]
   uint8_t* sV = sK + KST * TR::KV_BYTES;           // [VST][KV_BYTES]
@@ -207,21 +190,19 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* v_empty = v_full + VST;
   uint64_t* q_full = v_empty + VST;   // [2]
   uint64_t* q_empty = q_full + 2;     // [2]
-  uint64_t* s_full = q_empty + 2;     // [2] S_w holds a new tile
-  uint64_t* s_free = s_full + 2;      // [2] the softmax has read S_w
-  uint64_t* p_ready = s_free + 2;     // [2] P_w is in TMEM (and O rescaled if needed)
-  uint64_t* o_done = p_ready + 2;     // [2] a P_w V MMA group has completed
-  uint64_t* m_pub = o_done + 2;       // [2] warpgroup w published its tile's running max
-  uint64_t* b_ready = m_pub + 2;      // warpgroup B's row sums of the piece are in smem
-  uint64_t* merged = b_ready + 1;     // warpgroup A has read O of the piece
+  uint64_t* s_full = q_empty + 2;     // [2] per softmax warpgroup
+  uint64_t* p_ready = s_full + 2;     // [2]
+  uint64_t* o_done = p_ready + 2;     // [2]
+  uint64_t* b_ready = o_done + 2;     // warpgroup B's piece state is in smem
+  uint64_t* merged = b_ready + 1;     // warpgroup A has read O_A, O_B of the piece
   uint64_t* drain = merged + 1;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* q_tma = drain + 1;        // [2] TMA copy of a Q tile landed
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(q_tma + 2);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   volatile int* s_last = reinterpret_cast<volatile int*>(s_tmem + 2);
-  float* s_m = reinterpret_cast<float*>(ctrl + 384);        // [2][128] running max handed between warpgroups
-  float* s_lB = s_m + 2 * BM;                              // [128] warpgroup B's row sums at the end of a piece
-  float* s_mB = s_lB + BM;                                 // [128] ... and the max they are relative to
-  float* s_omega = s_mB + BM;                              // [2][D/2]: one head per Q buffer
+  float* s_mB = reinterpret_cast<float*>(ctrl + 384);      // [128]
+  float* s_lB = s_mB + BM;                                 // [128]
+  float* s_omega = reinterpret_cast<float*>(ctrl + 1408);  // [2][D/2]: one head per Q buffer
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.x;
@@ -241,14 +222,14 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], BM);
       mbar_init(&p_ready[s], BM);
       mbar_init(&o_done[s], 1);
-      mbar_init(&m_pub[s], BM);
     }
     mbar_init(b_ready, BM);
     mbar_init(merged, BM);
     mbar_init(drain, 1);
+    mbar_init(&q_tma[0], 1);
+    mbar_init(&q_tma[1], 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -272,18 +253,22 @@ __global__ void __launch_bounds__(384, 1)
     return true;
   };
 
-  // The first piece's Q is loaded by warps 2-11 together (the softmax
-  // warpgroups have nothing to do before it); later pieces by warps 2-3.
+  // The first piece's Q tile comes in by TMA; warps 2-11 rotate it together
+  // (the softmax warpgroups have nothing to do before it). Later pieces:
+  // warps 2-3.
   {
     long long it0 = it_begin;
     Piece pc0;
     next_piece(it0, pc0);
     if (warp >= 2) {
       const int tid = threadIdx.x - 64;  // 0..319
+      if (tid == 0) tma_q_tile<TR>(sQ, &tmQ, &q_tma[0], p, pc0.u);
       if (p.rp.enabled)
         for (int j = tid; j < D / 2; j += 320) s_omega[j] = omega_of(p.rp, (pc0.u / p.q_tiles) % p.H, j);
       asm volatile("bar.sync 4, 320;" ::: "memory");
-      load_q_tile<TR, 4>(sQ, p, s_omega, pc0.u, tid, 320);
+      const bool landed = mbar_wait(&q_tma[0], 0, s_abort);
+      if (landed && p.rp.enabled) rope_q_tile_inplace<TR>(sQ, p, s_omega, pc0.u, tid, 320);
+      if (!landed && tid == 0) mbar_wait_teardown(&q_tma[0], 0);  // the copy must land before the CTA exits
       asm volatile("bar.sync 4, 320;" ::: "memory");
       if (tid == 0) mbar_arrive(&q_full[0]);
     }
@@ -363,111 +348,78 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (event driven)
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_dense(BM, BN, TR::FMT, false, false);
       constexpr uint32_t idO = idesc_dense(BM, D, TR::FMT, false, true);
       const uint32_t aQ = smem_addr(sQ), aK = smem_addr(sK), aV = smem_addr(sV);
+      long long it = it_begin;
+      Piece pc;
+      int kc = 0, vc = 0, pidx = 0;
+      bool ok = true;
       // descriptor words of every buffer, computed once; an MMA then only adds
       // a constant to the low word
       const DescWords dQ = desc_words(aQ, 16, 1024, 2), dK = desc_words(aK, 16, 1024, 2);
       const DescWords dV = TR::ES == 2 ? desc_words(aV, BN * 128, 1024, 2) : desc_words(aV, BN * 128, 512, 1);
-      const uint32_t tO = tbase + TR::O_COL;
-      long long it = it_begin;
-      Piece pc;
-      int kc = 0, vc = 0, pidx = 0;
-      int s_iss0 = 0, s_iss1 = 0;  // S tiles issued into S_0 / S_1 so far
-      int pv_iss0 = 0, pv_iss1 = 0;  // P_0 V / P_1 V groups issued so far
-      bool ok = true;
+      auto issue_s = [&](int w, int qb) -> bool {
+        const int st = kc % KST;
+        if (!mbar_wait(&k_full[st], (kc / KST) & 1, s_abort)) return false;
+        tc_fence_after();
+        const uint32_t d = tbase + TR::S_COL0 + w * BN;
+        const uint32_t qoff = qb * TR::Q_BYTES, koff = st * TR::KV_BYTES;
+#pragma unroll
+        for (int k = 0; k < TR::QK_STEPS; ++k) {
+          const uint32_t off = (k >> 2) * (BM * 128) + (k & 3) * 32;
+          const uint32_t offk = (k >> 2) * (BN * 128) + (k & 3) * 32;
+          const uint64_t da = desc_at(dQ, qoff + off);
+          const uint64_t db = desc_at(dK, koff + offk);
+          if constexpr (TR::ES == 2) mma_bf16_ss(d, da, db, idS, k > 0 ? 1u : 0u);
+          else mma_tf32_ss(d, da, db, idS, k > 0 ? 1u : 0u);
+        }
+        mma_commit(&s_full[w]);
+        mma_commit(&k_empty[st]);
+        ++kc;
+        return true;
+      };
+      auto issue_pv = [&](int w, bool acc) {
+        const int st = vc % VST;
+        const uint32_t d = tbase + TR::O_COL0 + w * D;
+        const uint32_t pa = tbase + TR::S_COL0 + w * BN;  // P_w aliases S_w
+        const uint32_t voff = st * TR::KV_BYTES;
+#pragma unroll
+        for (int k = 0; k < TR::PV_STEPS; ++k) {
+          const uint64_t db = desc_at(dV, voff + k * TR::MMA_K * 128);
+          if constexpr (TR::ES == 2) mma_bf16_ts(d, pa + k * 8, db, idO, (acc || k > 0) ? 1u : 0u);
+          else mma_tf32_ts(d, pa + k * 8, db, idO, (acc || k > 0) ? 1u : 0u);
+        }
+        mma_commit(&o_done[w]);
+        mma_commit(&v_empty[st]);
+        ++vc;
+      };
+      int pcnt[2] = {0, 0};  // P tiles consumed per softmax warpgroup
       while (ok && next_piece(it, pc)) {
         const int qb = pidx & 1;
         ok = mbar_wait(&q_full[qb], (pidx >> 1) & 1, s_abort);
-        tc_fence_after();
-        int ns = 0, np = 0;  // next S / P V tile of the piece
-        long long idle_since = 0;
-        int polls = 0;
-        while (ok && np < pc.n) {
-          bool progressed = false;
-          if (ns < pc.n) {
-            const int w = ns & 1;
-            const int si = w ? s_iss1 : s_iss0, pi = w ? pv_iss1 : pv_iss0;
-            bool free_ok;
-            if (si == 0) free_ok = true;
-            else if (TR::P_SEPARATE) free_ok = mbar_test(smem_addr(&s_free[w]), (si - 1) & 1);
-            else free_ok = pi >= si;  // P aliases S: its P V must have been issued
-            if (free_ok && mbar_test(smem_addr(&k_full[kc % KST]), (kc / KST) & 1)) {
-              tc_fence_after();
-              const int st = kc % KST;
-              const uint32_t d = tbase + w * BN;
-              const uint32_t qoff = qb * TR::Q_BYTES, koff = st * TR::KV_BYTES;
-#pragma unroll
-              for (int k = 0; k < TR::QK_STEPS; ++k) {
-                const uint32_t off = (k >> 2) * (BM * 128) + (k & 3) * 32;
-                const uint32_t offk = (k >> 2) * (BN * 128) + (k & 3) * 32;
-                if constexpr (TR::ES == 2)
-                  mma_bf16_ss(d, desc_at(dQ, qoff + off), desc_at(dK, koff + offk), idS, k > 0 ? 1u : 0u);
-                else
-                  mma_tf32_ss(d, desc_at(dQ, qoff + off), desc_at(dK, koff + offk), idS, k > 0 ? 1u : 0u);
-              }
-              mma_commit(&s_full[w]);
-              mma_commit(&k_empty[st]);
-              ++kc;
-              if (w) ++s_iss1;
-              else ++s_iss0;
-              ++ns;
-              if (ns == pc.n) mma_commit(&q_empty[qb]);  // the piece's Q is no longer read
-              progressed = true;
-            }
-          }
-          if (np < ns) {
-            const int w = np & 1;
-            const int pi = w ? pv_iss1 : pv_iss0;
-            const bool ready = mbar_test(smem_addr(&p_ready[w]), pi & 1) &&
-                               (np != 0 || pidx == 0 || mbar_test(smem_addr(merged), (pidx - 1) & 1)) &&
-                               mbar_test(smem_addr(&v_full[vc % VST]), (vc / VST) & 1);
-            if (ready) {
-              tc_fence_after();
-              const int st = vc % VST;
-              const uint32_t pa = tbase + TR::P_COL0 + w * TR::P_STRIDE;
-              const uint32_t voff = st * TR::KV_BYTES;
-#pragma unroll
-              for (int k = 0; k < TR::PV_STEPS; ++k) {
-                const uint64_t db = desc_at(dV, voff + k * TR::MMA_K * 128);
-                if constexpr (TR::ES == 2) mma_bf16_ts(tO, pa + k * 8, db, idO, (np > 0 || k > 0) ? 1u : 0u);
-                else mma_tf32_ts(tO, pa + k * 8, db, idO, (np > 0 || k > 0) ? 1u : 0u);
-              }
-              mma_commit(&o_done[w]);
-              mma_commit(&v_empty[st]);
-              ++vc;
-              if (w) ++pv_iss1;
-              else ++pv_iss0;
-              ++np;
-              progressed = true;
-            }
-          }
-          if (progressed) {
-            idle_since = 0;
-            polls = 0;
-          } else if (++polls >= 64) {  // bounded: give up if nothing moves for ~1 s
-            polls = 0;
-            if (*s_abort) ok = false;
-            const long long now = clock64();
-            if (idle_since == 0) idle_since = now;
-            else if (now - idle_since > kWaitLimitCycles) {
-              atomicOr(&g_error_word, kErrWaitTimeout);
-              *s_abort = 1;
-              ok = false;
-            }
-          }
+        for (int i = 0; ok && i < 2 && i < pc.n; ++i) ok = issue_s(i, qb);
+        for (int i = 0; ok && i < pc.n; ++i) {
+          const int w = i & 1;
+          if (!mbar_wait(&p_ready[w], pcnt[w] & 1, s_abort)) { ok = false; break; }
+          ++pcnt[w];
+          // the previous piece's O_A / O_B must have been read before the first P V overwrites them
+          if (i == 0 && pidx > 0 && !mbar_wait(merged, (pidx - 1) & 1, s_abort)) { ok = false; break; }
+          if (!mbar_wait(&v_full[vc % VST], (vc / VST) & 1, s_abort)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(w, i >= 2);
+          if (i + 2 < pc.n && !issue_s(w, qb)) { ok = false; break; }
         }
-        if (ns < pc.n) mma_commit(&q_empty[qb]);  // aborted mid-piece
+        mma_commit(&q_empty[qb]);  // Q buffer free once every MMA issued so far has completed
         ++pidx;
       }
       mma_commit(drain);  // every MMA issued above has finished once `drain` completes
       mbar_wait_teardown(drain, 0);
     }
   } else {
-    // ------------------------------------------------ Q loader (warps 2-3) with fused RoPE
+    // ------------------------------------------------ Q loader (warps 2-3): TMA, then RoPE in place
     const int tid = threadIdx.x - 64;  // 0..63
     long long it = it_begin;
     Piece pc;
@@ -476,12 +428,17 @@ __global__ void __launch_bounds__(384, 1)
     while (next_piece(it, pc)) {
       const int qb = pidx & 1;
       const int h = (pc.u / p.q_tiles) % p.H;
-      const bool ok = mbar_wait(&q_empty[qb], ((pidx >> 1) & 1) ^ 1, s_abort);
+      bool ok = mbar_wait(&q_empty[qb], ((pidx >> 1) & 1) ^ 1, s_abort);
+      if (ok && tid == 0) tma_q_tile<TR>(sQ + qb * TR::Q_BYTES, &tmQ, &q_tma[qb], p, pc.u);
       float* om = s_omega + qb * (D / 2);
       if (ok && p.rp.enabled)
         for (int j = tid; j < D / 2; j += 64) om[j] = omega_of(p.rp, h, j);
       asm volatile("bar.sync 2, 64;" ::: "memory");
-      if (ok) load_q_tile<TR, 2>(sQ + qb * TR::Q_BYTES, p, om, pc.u, tid, 64);
+      if (ok) {
+        const bool landed = mbar_wait(&q_tma[qb], (pidx >> 1) & 1, s_abort);
+        if (landed && p.rp.enabled) rope_q_tile_inplace<TR>(sQ + qb * TR::Q_BYTES, p, om, pc.u, tid, 64);
+        if (!landed && tid == 0) mbar_wait_teardown(&q_tma[qb], (pidx >> 1) & 1);  // let the copy land
+      }
       asm volatile("bar.sync 2, 64;" ::: "memory");
       if (tid == 0) mbar_arrive(&q_full[qb]);
       ++pidx;
@@ -491,94 +448,86 @@ __global__ void __launch_bounds__(384, 1)
     // ------------------------------------------------ softmax warpgroups A (warps 4-7) and B (8-11)
     regs_inc<TR::REGS_HIGH>();
     const int wg = (warp - 4) >> 2;                // 0 = A, 1 = B
-    const int og = wg ^ 1;                         // the other warpgroup
     const int row = (threadIdx.x - 128) & 127;     // TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tbase + lane_off + wg * BN;
-    const uint32_t tP = tbase + lane_off + TR::P_COL0 + wg * TR::P_STRIDE;
-    const uint32_t tO = tbase + lane_off + TR::O_COL;
+    const uint32_t tS = tbase + lane_off + TR::S_COL0 + wg * BN;
+    const uint32_t tOA = tbase + lane_off + TR::O_COL0;
+    const uint32_t tOB = tOA + D;
+    const uint32_t tO = wg ? tOB : tOA;
     const float scale = p.softmax_scale > 0.f ? p.softmax_scale : rsqrtf(static_cast<float>(D));
     const float sl2 = scale * 1.4426950408889634f;
     long long it = it_begin;
     Piece pc;
-    int c_me = 0, c_ot = 0;  // tiles processed by this / the other warpgroup before the current piece
-    int pidx = 0;
+    int cnt = 0, pidx = 0;
     bool ok = true;
     while (next_piece(it, pc)) {
-      float l_w = 0.f;           // this warpgroup's row sum ...
-      float m_w = -INFINITY;     // ... relative to this max
-      float m_cur = -INFINITY;   // running max after this warpgroup's latest tile
-      for (int i = wg; i < pc.n; i += 2) {
-        const int k = c_me + (i >> 1);  // this tile's index among the warpgroup's tiles
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], k & 1, s_abort));
+      float m_run = -INFINITY, l_run = 0.f;
+      int mine = 0;
+      for (int i = wg; i < pc.n; i += 2, ++mine) {
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], cnt & 1, s_abort));
         if (!ok) continue;
         tc_fence_after();
         uint32_t sr[BN / 32][32];
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) tmem_load32(tS + c * 32, sr[c]);
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) tmem_load_wait(sr[c]);
-        // S_w may take the next tile now
-        tc_fence_before();
-        mbar_arrive(&s_free[wg]);
+        constexpr int HC = BN / 64;  // chunks of 32 columns per half
         const int kv_valid = p.Nk - (pc.j0 + i) * BN;
-        if (kv_valid < BN) {
-#pragma unroll
-          for (int c = 0; c < BN / 32; ++c)
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (c * 32 + e >= kv_valid) sr[c][e] = __float_as_uint(-INFINITY);
-        }
-        // row max: 3-input max over 8 independent chains (exact in any order)
+        // row max: 3-input max over 8 independent chains (exact in any order);
+        // the second half of S is loaded while the first half is reduced
         float mx8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c)
+        for (int c = 0; c < HC; ++c) tmem_load32(tS + c * 32, sr[c]);
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            mx8[e & 7] = fmax3(mx8[e & 7], __uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1]));
-        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
-        // the running max after the previous tile (the other warpgroup's)
-        float m_prev = -INFINITY;
-        int kp = -1;  // the previous tile's index among the other warpgroup's tiles
-        if (i > 0) {
-          kp = c_ot + ((i - 1) >> 1);
-          if (!__all_sync(0xffffffffu, mbar_wait(&m_pub[og], kp & 1, s_abort))) { ok = false; continue; }
-          m_prev = s_m[og * BM + row];
+        for (int c = 0; c < HC; ++c) tmem_load_wait(sr[c]);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          if (hf == 0) {
+#pragma unroll
+            for (int c = HC; c < 2 * HC; ++c) tmem_load32(tS + c * 32, sr[c]);
+          } else {
+#pragma unroll
+            for (int c = HC; c < 2 * HC; ++c) tmem_load_wait(sr[c]);
+          }
+          if (kv_valid < BN) {
+#pragma unroll
+            for (int c = hf * HC; c < (hf + 1) * HC; ++c)
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (c * 32 + e >= kv_valid) sr[c][e] = __float_as_uint(-INFINITY);
+          }
+#pragma unroll
+          for (int c = hf * HC; c < (hf + 1) * HC; ++c)
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              mx8[e & 7] = fmax3(mx8[e & 7], __uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1]));
         }
+        const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
         const float m_new = mx * sl2;
-        const float m_i = (m_new > m_prev + 8.0f) ? m_new : m_prev;  // lazy: move only on a 2^8 jump
-        s_m[wg * BM + row] = m_i;
-        mbar_arrive(&m_pub[wg]);
-        // O holds the P V of tiles up to i-1 relative to m_prev: bring it to m_i
-        const bool rescale = (i > 0) && (m_i > m_prev);
+        float m_use = m_run;
+        bool rescale = false;
+        if (m_new > m_run + 8.0f) {
+          m_use = m_new;
+          rescale = (mine > 0);
+        }
+        // S_i complete implies this warpgroup's previous P V (issued before it) is complete
         if (__any_sync(0xffffffffu, rescale)) {
-          if (!__all_sync(0xffffffffu, mbar_wait(&o_done[og], kp & 1, s_abort))) { ok = false; continue; }
-          tc_fence_after();
-          const float alpha = rescale ? ex2(m_prev - m_i) : 1.0f;
+          const float alpha = rescale ? ex2(m_run - m_use) : 1.0f;
+          l_run *= alpha;
 #pragma unroll 1
-          for (int c = 0; c < D / 16; ++c) {
-            uint32_t o[16];
-            tmem_load16(tO + c * 16, o);
-            tmem_load_wait16(o);
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_load32(tO + c * 32, o);
+            tmem_load_wait(o);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_store16(tO + c * 16, o);
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_store32(tO + c * 32, o);
           }
         }
-        // this warpgroup's own sum follows the max it is relative to
-        if (m_w != m_i) {
-          l_w *= ex2(m_w - m_i);
-          m_w = m_i;
-        }
-        m_cur = m_i;
-        // P_w is free once this warpgroup's previous P V has completed
-        if (k > 0 && !__all_sync(0xffffffffu, mbar_wait(&o_done[wg], (k - 1) & 1, s_abort))) { ok = false; continue; }
+        m_run = m_use;
         // p = 2^(s * scale * log2(e) - m) on pairs: the argument with one packed
         // FMA, the exponential on the MUFU unit (optionally some pairs on the FMA
         // pipe), the running sum in 4 packed partial sums
-        const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_i, -m_i);
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_use, -m_use);
         uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
@@ -603,38 +552,39 @@ __global__ void __launch_bounds__(384, 1)
               sr[c][2 * e + 1] = __float_as_uint(a2);
             }
           }
-          if constexpr (TR::ES == 2) tmem_store16(tP + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[c][0]));
-          else tmem_store32(tP + c * 32, sr[c]);
+          if constexpr (TR::ES == 2) tmem_store16(tS + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[c][0]));
+          else tmem_store32(tS + c * 32, sr[c]);
         }
         {
           const uint64_t s01 = f2_add(f2_add(ls2[0], ls2[1]), f2_add(ls2[2], ls2[3]));
           float u0, u1;
           f2_unpack(s01, u0, u1);
-          l_w += u0 + u1;
+          l_run += u0 + u1;
         }
         tmem_store_wait();
         tc_fence_before();
         mbar_arrive(&p_ready[wg]);
+        ++cnt;
       }
-      const int mine = (pc.n - wg + 1) / 2;  // tiles of this warpgroup in the piece
-      // ---- end of the piece
+      // ---- end of the piece: the last P V of this warpgroup must be complete
+      if (mine > 0 && ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_done[wg], (cnt - 1) & 1, s_abort));
       if (wg == 1) {
-        // B: hand its row sums over to A once A is done with the previous piece
+        // B: hand (m, l) over to A once A is done with the previous piece
         if (pidx > 0 && ok) ok = __all_sync(0xffffffffu, mbar_wait(merged, (pidx - 1) & 1, s_abort));
-        s_lB[row] = mine > 0 ? l_w : 0.f;
-        s_mB[row] = mine > 0 ? m_cur : -INFINITY;
+        s_mB[row] = mine > 0 ? m_run : -INFINITY;
+        s_lB[row] = mine > 0 ? l_run : 0.f;
+        tc_fence_before();
         mbar_arrive(b_ready);
       } else {
-        // A: wait for B's sums and for the piece's last P V, then write O (whole
-        // unit) or a partial
+        // A: merge the two halves, then write O (whole unit) or a partial
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(b_ready, pidx & 1, s_abort));
-        const int wl = (pc.n - 1) & 1;                       // warpgroup of the last tile
-        const int kl = (wl == wg ? c_me : c_ot) + ((pc.n - 1) >> 1);  // its index among that warpgroup's tiles
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_done[wl], kl & 1, s_abort));
         tc_fence_after();
+        const bool hasB = pc.n >= 2;
         const float mB = s_mB[row], lB = s_lB[row];
-        const float mm = fmaxf(m_cur, mB);                   // the max of the piece's last tile
-        const float L = l_w * ex2(m_w - mm) + (lB > 0.f ? lB * ex2(mB - mm) : 0.f);
+        const float mm = fmaxf(m_run, mB);
+        const float aA = ex2(m_run - mm);
+        const float aB = hasB ? ex2(mB - mm) : 0.f;
+        const float L = l_run * aA + lB * aB;
         const int qt = pc.u % p.q_tiles;
         const int h = (pc.u / p.q_tiles) % p.H;
         const int b = pc.u / (p.q_tiles * p.H);
@@ -647,16 +597,23 @@ __global__ void __launch_bounds__(384, 1)
         const float inv_L = 1.0f / L;
         if (ok) {
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_load32(tO + c * 32, o);
-            tmem_load_wait(o);
-            const float* x = reinterpret_cast<const float*>(o);
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t oa[16], ob[16];
+            tmem_load16(tOA + c * 16, oa);
+            tmem_load_wait16(oa);
+            if (hasB) {
+              tmem_load16(tOB + c * 16, ob);
+              tmem_load_wait16(ob);
+            }
+            float* x = reinterpret_cast<float*>(oa);  // merged in place
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              x[e] = __uint_as_float(oa[e]) * aA + (hasB ? __uint_as_float(ob[e]) * aB : 0.f);
             if (whole) {
               if (t < p.Tq) {
-                T* dst = static_cast<T*>(p.out) + ((static_cast<size_t>(b) * p.Tq + t) * p.H + h) * D + c * 32;
+                T* dst = static_cast<T*>(p.out) + ((static_cast<size_t>(b) * p.Tq + t) * p.H + h) * D + c * 16;
 #pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
+                for (int q8 = 0; q8 < 2; ++q8) {
                   float y[8];
 #pragma unroll
                   for (int e = 0; e < 8; ++e) y[e] = x[q8 * 8 + e] * inv_L;
@@ -664,15 +621,15 @@ __global__ void __launch_bounds__(384, 1)
                 }
               }
             } else {
-              float4* dst = reinterpret_cast<float4*>(slot + static_cast<size_t>(row) * D + c * 32);
+              float4* dst = reinterpret_cast<float4*>(slot + static_cast<size_t>(row) * D + c * 16);
 #pragma unroll
-              for (int q4 = 0; q4 < 8; ++q4)
+              for (int q4 = 0; q4 < 4; ++q4)
                 dst[q4] = make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]);
             }
           }
         }
         tc_fence_before();
-        mbar_arrive(merged);  // O and s_lB / s_mB may be reused
+        mbar_arrive(merged);  // O_A, O_B and s_mB / s_lB may be reused
         if (whole) {
           if (ok && p.lse != nullptr && t < p.Tq)
             p.lse[(static_cast<size_t>(b) * p.H + h) * p.Tq + t] = (mm + log2f(L)) * 0.6931471805599453f;
@@ -723,8 +680,6 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
-      c_me += (pc.n + 1 - wg) / 2;  // warpgroup A takes the even tiles, B the odd ones
-      c_ot += (pc.n + wg) / 2;
       ++pidx;
     }
   }
