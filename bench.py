@@ -562,6 +562,37 @@ def run_attention_only(args):
             "frac_of_burst_peak": round(fl / t / 1e12 / peaks["bf16_tflops"], 4), "peak_kind": kind}
 
 
+def run_append_only(args):
+    """One Wan frame's RoPE + append into a layer cache (bf16 or E4M3 cache):
+    `warmup` + `steps` launches, each after a 256 MB write that evicts L2,
+    timed with CUDA events; achieved HBM bandwidth from the algorithmic bytes."""
+    from sink_window_attention_b200 import build
+    build.build()
+    import sink_window_attention_b200 as swa
+    w = W.WAN
+    st = Stream(W.replace(w, layers=1, sigma_t=0.8, jitter_seed=4), args.cache, "cuda")
+    flush = torch.empty(64 << 20, dtype=torch.float32, device="cuda")
+    f0 = 3 * 40
+    ev = []
+    for i in range(args.warmup + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush.zero_()
+        torch.cuda._sleep(200_000)
+        a.record()
+        swa.kvcache_append(st.caches[0], st.k[0][i % POOL], st.v[0][i % POOL], f0 + i, st.rope)
+        b.record()
+        ev.append((a, b))
+    torch.cuda.synchronize()
+    times = [a.elapsed_time(b) / 1e3 for a, b in ev[args.warmup:]]
+    assert swa.device_error() == 0
+    nbytes = append_bytes(w, 1 if args.cache == "fp8" else 2)
+    peaks, kind = measured_peaks()
+    t = statistics.median(times)
+    return {"mode": "append", "cache": args.cache, "launches": len(times), "median_us": round(t * 1e6, 2),
+            "algorithmic_bytes": nbytes, "gbs": round(nbytes / t / 1e9, 1),
+            "frac_of_hbm_peak": round(nbytes / t / 1e9 / peaks["hbm_gbs"], 4), "peak_kind": kind}
+
+
 def run_recache_only(args):
     """One layer's KV recache at the Wan shape (X [18720, 1536], Wk, Wv
     [1536, 1536]): `warmup` + `steps` launches timed with CUDA events."""
@@ -599,7 +630,7 @@ def main():
     ap.add_argument("--layers", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
-    ap.add_argument("--mode", default="stream", choices=["stream", "attention", "recache"])
+    ap.add_argument("--mode", default="stream", choices=["stream", "attention", "recache", "append"])
     ap.add_argument("--workload", default="wan", choices=["wan", "chunk"])
     args = ap.parse_args()
     if args.mode == "attention":
@@ -607,6 +638,9 @@ def main():
         return
     if args.mode == "recache":
         print(json.dumps(run_recache_only(args)), flush=True)
+        return
+    if args.mode == "append":
+        print(json.dumps(run_append_only(args)), flush=True)
         return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

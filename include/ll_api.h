@@ -89,6 +89,8 @@ typedef struct ll_rope_desc {
  * k, v: [B][S*N][H][D] of `dtype` (F32, BF16 or FP8_E4M3).
  * k_scale, v_scale: [B][S*N][H] fp32 dequantisation scales, FP8 only
  * (value = decode(code) * scale); NULL for the other dtypes.
+ * D: a multiple of 16; an FP8 cache needs D = 16 * 2^k <= 256
+ * (LL_ERR_UNSUPPORTED otherwise). k and v must be 16-byte aligned.
  */
 typedef struct ll_kvcache {
   void* k;

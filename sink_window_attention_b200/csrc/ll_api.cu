@@ -86,6 +86,11 @@ ll_status check_cache(const ll_kvcache* c) {
     return fail(LL_ERR_INVALID_ARG, "cache sizes must be positive (B=%d H=%d D=%d N=%d)", c->B, c->H, c->D,
                 c->tokens_per_frame);
   if (c->D % 16 != 0) return fail(LL_ERR_INVALID_ARG, "D = %d must be a multiple of 16", c->D);
+  if (c->dtype == LL_FP8_E4M3) {  // a row's max|x| is reduced over its D / 8 lanes: a power of two up to 32
+    const int lanes = c->D / 8;
+    if ((lanes & (lanes - 1)) != 0 || lanes > 32)
+      return fail(LL_ERR_UNSUPPORTED, "an FP8 cache needs D = 16 * 2^k <= 256 (got D = %d)", c->D);
+  }
   if (c->H > ll::kMaxHeads) return fail(LL_ERR_INVALID_ARG, "H = %d exceeds %d", c->H, ll::kMaxHeads);
   if (c->n_sink < 0 || c->n_local < 1) return fail(LL_ERR_INVALID_ARG, "need n_sink >= 0 and n_local >= 1");
   return LL_OK;
@@ -303,11 +308,16 @@ ll_status ll_kvcache_append(const ll_kvcache* cache, const void* k, const void* 
   p.first_frame = first_frame;
   if (slots_out)
     for (int i = 0; i < n_frames; ++i) ll_slot_of_frame(first_frame + i, cache->n_sink, cache->n_local, &slots_out[i]);
-  const long long chunks = static_cast<long long>(p.B) * n_frames * p.N * p.H * (p.D / 8);
-  if (chunks >= (1LL << 31)) return fail(LL_ERR_UNSUPPORTED, "tensor too large for one call (%lld chunks)", chunks);
-  const long long want = (chunks + 255) / 256;
+  // threads: one per (token, 8-element chunk, group of append_heads_per_thread(H) heads)
+  const long long threads = static_cast<long long>(p.B) * n_frames * p.N * (p.D / 8) *
+                            (p.H / ll::append_heads_per_thread(p.H));
+  if (threads >= (1LL << 31)) return fail(LL_ERR_UNSUPPORTED, "tensor too large for one call (%lld threads)", threads);
+  const long long want = (threads + 255) / 256;
   const int grid = static_cast<int>(want < 8LL * num_sms() ? want : 8LL * num_sms());
-  const size_t smem = static_cast<size_t>(p.H) * (p.D / 2) * sizeof(float);
+  const size_t smem = ll::append_smem_bytes(n_frames, p.H, p.D, p.rp.pt);
+  if (smem > 48 * 1024)
+    return fail(LL_ERR_UNSUPPORTED, "frequency tables of %zu bytes exceed 48 KiB (n_frames x H x pairs_t too large)",
+                smem);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cache->dtype == LL_BF16)
     ll::append_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 256, smem, s>>>(p);

@@ -29,21 +29,19 @@ struct RopeParams {
 // omega_i = base^(-2i/d) for pair j = 0..P-1 of head h (P = D/2): the temporal
 // band (j < pt) uses base theta0 (1 + sigma eps_h), the row and column bands
 // theta0; inside a band of `pairs` pairs, d = 2 * pairs. Evaluated in fp32 as
-// exp2(-(i/pairs) * log2(base)): the relative error of omega is below 1e-6,
-// i.e. under 3e-4 rad of angle at position 3000, far below bf16 resolution.
+// exp2(-(i/pairs) * log2(base)) (base itself in fp32: 6e-8 relative): the
+// relative error of omega is below 1e-6, i.e. under 3e-4 rad of angle at
+// position 3000, far below bf16 resolution.
 __device__ __forceinline__ float omega_of(const RopeParams& rp, int h, int j) {
-  float base;
-  int i, pairs;
+  const float theta0 = static_cast<float>(rp.theta0);
+  float base = theta0;
+  int i = j, pairs = rp.pt;
   if (j < rp.pt) {
-    base = static_cast<float>(rp.theta0 * (1.0 + rp.sigma * static_cast<double>(rp.eps[h])));
-    i = j;
-    pairs = rp.pt;
+    base = theta0 * fmaf(static_cast<float>(rp.sigma), rp.eps[h], 1.0f);
   } else if (j < rp.pt + rp.ph) {
-    base = static_cast<float>(rp.theta0);
     i = j - rp.pt;
     pairs = rp.ph;
   } else {
-    base = static_cast<float>(rp.theta0);
     i = j - rp.pt - rp.ph;
     pairs = rp.pw;
   }
@@ -64,26 +62,12 @@ __device__ __forceinline__ void build_omega_one_head(float* omega, const RopePar
   for (int j = tid; j < P; j += nthreads) omega[j] = omega_of(rp, h, j);
 }
 
-// Rotate the 4 pairs (x[0],x[1]) .. (x[6],x[7]) whose first pair index is j0
-// with [[cos, -sin], [sin, cos]] at angle pos_axis * omega_j.
-__device__ __forceinline__ void rotate_chunk8(float (&x)[8], int j0, float pos_t, float pos_r, float pos_c,
-                                              const float* omega_h, int pt, int pth) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int j = j0 + q;
-    const float pos = j < pt ? pos_t : (j < pth ? pos_r : pos_c);
-    float s, c;
-    sincosf(pos * omega_h[j], &s, &c);
-    const float a = x[2 * q], b = x[2 * q + 1];
-    x[2 * q] = a * c - b * s;
-    x[2 * q + 1] = a * s + b * c;
-  }
-}
-
 // sin and cos of x for |x| up to ~1e5: Cody and Waite's two-constant
 // reduction x = k 2pi + r (k = rint(x / 2pi); 2pi split into its float
 // rounding and the remainder, each product taken in one FMA) brings r into
 // [-pi, pi], where the hardware approximation is accurate to ~4e-7 absolute.
+// (The fp32 angle pos * omega itself carries ~1e-4 rad of rounding at frame
+// indices in the thousands, far above either error.)
 __device__ __forceinline__ void sincos_reduced(float x, float& s, float& c) {
   const float k = rintf(x * 0.15915494309189535f);
   float r = fmaf(-k, 6.28318548202514648f, x);
@@ -91,9 +75,10 @@ __device__ __forceinline__ void sincos_reduced(float x, float& s, float& c) {
   __sincosf(r, &s, &c);
 }
 
-// rotate_chunk8 with sincos_reduced (query tiles staged by the attention kernel)
-__device__ __forceinline__ void rotate_chunk8_fast(float (&x)[8], int j0, float pos_t, float pos_r, float pos_c,
-                                                   const float* omega_h, int pt, int pth) {
+// Rotate the 4 pairs (x[0],x[1]) .. (x[6],x[7]) whose first pair index is j0
+// with [[cos, -sin], [sin, cos]] at angle pos_axis * omega_j.
+__device__ __forceinline__ void rotate_chunk8(float (&x)[8], int j0, float pos_t, float pos_r, float pos_c,
+                                              const float* omega_h, int pt, int pth) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const int j = j0 + q;
@@ -145,15 +130,9 @@ __device__ __forceinline__ void store_chunk8<float>(float* p, const float (&x)[8
   *reinterpret_cast<float4*>(p + 4) = make_float4(x[4], x[5], x[6], x[7]);
 }
 
-// E4M3 codes of x / scale for one chunk; the (token, head) row of D values is
-// spread over `group` consecutive lanes, which reduce max|x| with shuffles.
-__device__ __forceinline__ uint2 quantize_chunk8_e4m3(const float (&x)[8], int group, float* scale_out) {
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
-  for (int off = group >> 1; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  const float scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-  *scale_out = scale;
+// E4M3 codes of x / scale for one chunk of 8 values (IEEE fp32 quotient,
+// round to nearest even, saturating at +-448).
+__device__ __forceinline__ uint2 encode_chunk8_e4m3(const float (&x)[8], float scale) {
   uint32_t w[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -227,68 +206,162 @@ __device__ __forceinline__ int cache_slot(long long f, int n_sink, int n_local) 
   return f < n_sink ? static_cast<int>(f) : n_sink + static_cast<int>((f - n_sink) % n_local);
 }
 
+// One thread: one 8-element chunk position c of one token, for a group of
+// `hg` heads. The angles of the chunk's 4 pairs are shared: a pair of the row
+// or column band has the same angle in every head (no jitter there), and a
+// pair of the temporal band has the same angle for every token of a frame,
+// so its cos/sin come from a per-block table [F][H][pt]. Consecutive threads
+// take consecutive chunks of a (token, head) row, so every access is a
+// coalesced 16 bytes.
+__host__ __device__ __forceinline__ int append_heads_per_thread(int H) {
+  return (H % 4 == 0) ? 4 : (H % 3 == 0 ? 3 : (H % 2 == 0 ? 2 : 1));
+}
+constexpr int kAppendMaxHg = 4;
+
+__host__ __device__ __forceinline__ size_t append_smem_bytes(int F, int H, int D, int pt) {
+  return (static_cast<size_t>(H) * (D / 2) + 2 * static_cast<size_t>(F) * H * pt) * sizeof(float);
+}
+
 template <typename Tin, typename C>
 __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
-  extern __shared__ float s_omega[];  // [H][D/2]
+  extern __shared__ float s_tab[];      // omega [H][D/2], then cos, sin of the temporal band [F][H][pt][2]
   const int P = p.D / 2;
-  if (p.rp.enabled) build_omega(s_omega, p.rp, 0, p.H, P);
-  __syncthreads();
-  const int cpr = p.D / 8;
-  const int total = p.B * p.F * p.N * p.H * cpr;  // < 2^31, checked on the host
+  float* s_omega = s_tab;
+  float* s_tcs = s_tab + p.H * P;
+  const int cpr = p.D / 8;                        // chunks per (token, head) row
+  const int hg = append_heads_per_thread(p.H);    // heads per thread
+  const int ngroups = p.H / hg;
+  const int total = p.B * p.F * p.N * ngroups * cpr;  // < 2^31, checked on the host
   const int FN = p.F * p.N;
   const int S = p.n_sink + p.n_local;
   const int pth = p.rp.pt + p.rp.ph;
   const Tin* kin = static_cast<const Tin*>(p.k_in);
   const Tin* vin = static_cast<const Tin*>(p.v_in);
+  const int stride = gridDim.x * blockDim.x;
+  float kx[kAppendMaxHg][8], vx[kAppendMaxHg][8];
+  auto load = [&](int idx) {
+    const bool active = idx < total;
+    const int i = active ? idx : 0;
+    const int grow = i / cpr, c = i - grow * cpr;
+    const int bt = grow / ngroups;
+    const size_t src0 = (static_cast<size_t>(bt) * p.H + (grow - bt * ngroups) * hg) * p.D + c * 8;
+#pragma unroll
+    for (int k = 0; k < kAppendMaxHg; ++k) {
+      if (active && k < hg) {
+        load_chunk8<Tin>(kin + src0 + static_cast<size_t>(k) * p.D, kx[k]);
+        load_chunk8<Tin>(vin + src0 + static_cast<size_t>(k) * p.D, vx[k]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) kx[k][e] = vx[k][e] = 0.f;
+      }
+    }
+  };
+  // the first chunks' loads go out before the tables are built, so the
+  // table work overlaps their latency
+  int base = blockIdx.x * blockDim.x;
+  load(base + threadIdx.x);
+  if (p.rp.enabled) {
+    build_omega(s_omega, p.rp, 0, p.H, P);
+    __syncthreads();
+    const int nt = p.F * p.H * p.rp.pt;
+    for (int idx = threadIdx.x; idx < nt; idx += blockDim.x) {
+      const int f = idx / (p.H * p.rp.pt), rem = idx - f * (p.H * p.rp.pt);
+      const int h = rem / p.rp.pt, j = rem - h * p.rp.pt;
+      float sn, cs;
+      sincos_reduced(static_cast<float>(p.rp.t_first + f) * s_omega[h * P + j], sn, cs);
+      s_tcs[2 * idx] = cs;
+      s_tcs[2 * idx + 1] = sn;
+    }
+  }
+  __syncthreads();
   // All threads of the block run the same number of iterations, so the
   // shuffles of the FP8 path always see full warps.
-  for (int base = blockIdx.x * blockDim.x; base < total; base += gridDim.x * blockDim.x) {
+  for (; base < total; base += stride) {
     const int idx = base + threadIdx.x;
     const bool active = idx < total;
     const int i = active ? idx : 0;
-    const int row = i / cpr;
-    const int c = i - row * cpr;
-    const int bt = row / p.H;                       // b * F*N + tok
-    const int h = row - bt * p.H;
+    const int grow = i / cpr;                     // (b * F*N + tok) * ngroups + group
+    const int c = i - grow * cpr;
+    const int bt = grow / ngroups;
+    const int h0 = (grow - bt * ngroups) * hg;
     const int b = bt / FN;
     const int tok = bt - b * FN;
     const int fi = tok / p.N;
     const int n = tok - fi * p.N;
     const int slot = cache_slot(p.first_frame + fi, p.n_sink, p.n_local);
-    const size_t drow = (static_cast<size_t>(b) * S * p.N + static_cast<size_t>(slot) * p.N + n) * p.H + h;
-    float kx[8], vx[8];
-    if (active) {
-      load_chunk8<Tin>(kin + static_cast<size_t>(row) * p.D + c * 8, kx);
-      load_chunk8<Tin>(vin + static_cast<size_t>(row) * p.D + c * 8, vx);
-      if (p.rp.enabled) {
-        const int r = n / p.rp.grid_w, col = n - r * p.rp.grid_w;
-        rotate_chunk8(kx, c * 4, static_cast<float>(p.rp.t_first + fi), static_cast<float>(r),
-                      static_cast<float>(col), s_omega + h * P, p.rp.pt, pth);
-      }
-    } else {
+    const size_t dst0 = ((static_cast<size_t>(b) * S * p.N + static_cast<size_t>(slot) * p.N + n) * p.H + h0) * p.D +
+                        c * 8;
+    if (active && p.rp.enabled) {
+      const float pos_r = static_cast<float>(n / p.rp.grid_w), pos_c = static_cast<float>(n % p.rp.grid_w);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) kx[e] = vx[e] = 0.f;
+      for (int q = 0; q < 4; ++q) {
+        const int j = c * 4 + q;
+        float cs[kAppendMaxHg], sn[kAppendMaxHg];
+        if (j < p.rp.pt) {  // temporal band: per-head angle from the table
+#pragma unroll
+          for (int k = 0; k < kAppendMaxHg; ++k) {
+            const int e = k < hg ? ((fi * p.H + h0 + k) * p.rp.pt + j) : 0;
+            cs[k] = s_tcs[2 * e];
+            sn[k] = s_tcs[2 * e + 1];
+          }
+        } else {  // row / column band: one angle for all heads
+          float s1, c1;
+          sincos_reduced((j < pth ? pos_r : pos_c) * s_omega[j], s1, c1);
+#pragma unroll
+          for (int k = 0; k < kAppendMaxHg; ++k) {
+            cs[k] = c1;
+            sn[k] = s1;
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < kAppendMaxHg; ++k) {
+          const float x0 = kx[k][2 * q], x1 = kx[k][2 * q + 1];
+          kx[k][2 * q] = x0 * cs[k] - x1 * sn[k];
+          kx[k][2 * q + 1] = x0 * sn[k] + x1 * cs[k];
+        }
+      }
     }
     if constexpr (sizeof(C) == 1) {
-      float ks, vs;
-      const uint2 kq = quantize_chunk8_e4m3(kx, cpr, &ks);
-      const uint2 vq = quantize_chunk8_e4m3(vx, cpr, &vs);
-      if (active) {
-        uint8_t* kc = static_cast<uint8_t*>(p.k_cache);
-        uint8_t* vc = static_cast<uint8_t*>(p.v_cache);
-        *reinterpret_cast<uint2*>(kc + drow * p.D + c * 8) = kq;
-        *reinterpret_cast<uint2*>(vc + drow * p.D + c * 8) = vq;
-        if (c == 0) {
-          p.k_scale[drow] = ks;
-          p.v_scale[drow] = vs;
+      // per (token, head) row: scale = max|x| / 448 over the row's D values,
+      // which lie in the cpr consecutive lanes of this chunk position's group
+      uint8_t* kc = static_cast<uint8_t*>(p.k_cache) + dst0;
+      uint8_t* vc = static_cast<uint8_t*>(p.v_cache) + dst0;
+#pragma unroll
+      for (int k = 0; k < kAppendMaxHg; ++k) {
+        if (k >= hg) break;  // hg is uniform across the grid
+        float ka = 0.f, va = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          ka = fmaxf(ka, fabsf(kx[k][e]));
+          va = fmaxf(va, fabsf(vx[k][e]));
+        }
+        for (int off = cpr >> 1; off > 0; off >>= 1) {
+          ka = fmaxf(ka, __shfl_xor_sync(0xffffffffu, ka, off));
+          va = fmaxf(va, __shfl_xor_sync(0xffffffffu, va, off));
+        }
+        const float ks = ka > 0.f ? __fdiv_rn(ka, 448.0f) : 1.0f;
+        const float vs = va > 0.f ? __fdiv_rn(va, 448.0f) : 1.0f;
+        if (active) {
+          *reinterpret_cast<uint2*>(kc + static_cast<size_t>(k) * p.D) = encode_chunk8_e4m3(kx[k], ks);
+          *reinterpret_cast<uint2*>(vc + static_cast<size_t>(k) * p.D) = encode_chunk8_e4m3(vx[k], vs);
+          if (c == 0) {
+            const size_t srow = dst0 / p.D + k;
+            p.k_scale[srow] = ks;
+            p.v_scale[srow] = vs;
+          }
         }
       }
     } else {
       if (active) {
-        store_chunk8<C>(static_cast<C*>(p.k_cache) + drow * p.D + c * 8, kx);
-        store_chunk8<C>(static_cast<C*>(p.v_cache) + drow * p.D + c * 8, vx);
+#pragma unroll
+        for (int k = 0; k < kAppendMaxHg; ++k)
+          if (k < hg) {
+            store_chunk8<C>(static_cast<C*>(p.k_cache) + dst0 + static_cast<size_t>(k) * p.D, kx[k]);
+            store_chunk8<C>(static_cast<C*>(p.v_cache) + dst0 + static_cast<size_t>(k) * p.D, vx[k]);
+          }
       }
     }
+    if (base + stride < total) load(base + stride + threadIdx.x);  // uniform condition
   }
 }
 
