@@ -125,7 +125,7 @@ def test_append_fp8_codes_and_scales():
 
 # ---------------------------------------------------------------------------- attention
 def run_stream(w: W.Workload, frames, layer=0, rows_per_step=48, q_scale=1.0, check_lse=True, dtype=None,
-               B=None, mean_abs=1e-3, lse_rel=1e-3, max_rel=1e-2):
+               B=None, mean_abs=1e-3, lse_rel=1e-3, max_rel=1e-2, scale=None):
     """Append + attend frame by frame (or chunk by chunk); compare sampled rows
     (all rows when the step is small) with the oracle stream."""
     B = B or w.B
@@ -143,12 +143,12 @@ def run_stream(w: W.Workload, frames, layer=0, rows_per_step=48, q_scale=1.0, ch
             q = (q.float() * q_scale).to(q.dtype)
         swa.kvcache_append(cache, k.cuda(), v.cuda(), f0, rope)
         lse = torch.empty(B, w.H, q.shape[1], device="cuda", dtype=torch.float32)
-        out = swa.sink_window_attention(q.cuda(), cache, f0, rope, lse=lse)
+        out = swa.sink_window_attention(q.cuda(), cache, f0, rope, lse=lse, softmax_scale=scale or 0.0)
         Tq = q.shape[1]
         rows = np.arange(Tq) if Tq <= 256 else sample_rows(Tq, rows_per_step, f0)
         for b in range(B):
             oracles[b].append(f0, np64(k[b]), np64(v[b]))
-            ref, ref_lse = oracles[b].attend(np64(q[b]), f0, rows=rows, return_lse=True)
+            ref, ref_lse = oracles[b].attend(np64(q[b]), f0, scale=scale, rows=rows, return_lse=True)
             got = np64(out[b])[rows]
             r = assert_parity(got, ref, max_rel=max_rel, mean_abs=mean_abs, what=f"{w.name} frame {f0} b {b}")
             worst = (max(worst[0], r[0]), max(worst[1], r[1]))
@@ -206,3 +206,33 @@ def test_attention_fp8_cache(name, frames):
     unquantised fp64 reference, max|err| <= 5e-2 * max|ref|."""
     w = W.WORKLOADS[name]
     run_stream(w, frames, dtype="fp8", rows_per_step=24, mean_abs=5e-3, lse_rel=5e-3, max_rel=5e-2)
+
+
+def test_attention_chunk_d64_batch3():
+    """3-frame chunks at D = 64 (bf16), three independent streams in one call,
+    jitter and a temporal offset: 180 query rows per chunk (a full and a
+    ragged 52-row query tile), 720 keys (a ragged 80-key last tile); every
+    output row is checked."""
+    w = W.replace(W.CHUNK, name="chunk_d64", H=3, D=64, pairs=(12, 10, 10), grid_h=6, grid_w=10, t_offset=500)
+    run_stream(w, range(0, 18, 3), B=3)
+
+
+def test_attention_softmax_scale():
+    """A softmax scale other than 1/sqrt(D) reaches the kernel and the oracle."""
+    w = W.replace(W.TINY, dtype="bf16", name="tiny_bf16")
+    run_stream(w, range(14), scale=0.05)
+
+
+def test_attention_deterministic():
+    """The split of the key range over CTAs and the merge order are fixed, so
+    repeated launches on the same inputs give bit-identical outputs."""
+    w = W.WAN
+    cache = swa.KVCache(w.B, w.H, w.D, w.N, w.dtype)
+    rope = rope_of(w)
+    for f in range(13):
+        _, k, v = W.qkv_frames(w, 0, f, 1)
+        swa.kvcache_append(cache, k.cuda(), v.cuda(), f, rope)
+    q = W.qkv_frames(w, 0, 12, 1)[0].cuda()
+    outs = [swa.sink_window_attention(q, cache, 12, rope).clone() for _ in range(3)]
+    torch.cuda.synchronize()
+    assert all(torch.equal(outs[0], o) for o in outs[1:])
