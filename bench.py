@@ -533,7 +533,7 @@ def run_attention_only(args):
     build.build()
     import sink_window_attention_b200 as swa
     w = W.WAN if args.workload == "wan" else W.CHUNK
-    st = Stream(W.replace(w, layers=1, sigma_t=0.8, jitter_seed=4), "bf16", "cuda")
+    st = Stream(W.replace(w, layers=1, sigma_t=0.8, jitter_seed=4), args.cache, "cuda")
     c = w.query_frames
     q = W.normal((1, c * w.N, w.H, w.D), 99, w.qkv_scale, torch.bfloat16, "cuda")
     out = torch.empty_like(q)
@@ -557,7 +557,8 @@ def run_attention_only(args):
     fl = 4.0 * (c * w.N) * (w.slots * w.N) * w.D * w.H
     peaks, kind = measured_peaks()
     t = statistics.median(times)
-    return {"mode": "attention", "workload": w.name, "launches": len(times), "median_us": round(t * 1e6, 2),
+    return {"mode": "attention", "workload": w.name, "cache": args.cache, "launches": len(times),
+            "median_us": round(t * 1e6, 2),
             "min_us": round(min(times) * 1e6, 2), "tflops": round(fl / t / 1e12, 1),
             "frac_of_burst_peak": round(fl / t / 1e12 / peaks["bf16_tflops"], 4), "peak_kind": kind}
 

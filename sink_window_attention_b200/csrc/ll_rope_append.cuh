@@ -378,32 +378,54 @@ struct DequantParams {
 };
 
 __global__ void __launch_bounds__(256) dequant_e4m3_kernel(const DequantParams p) {
-  const int which = blockIdx.y;
+  constexpr int U = 4;  // chunks per thread per pass: their loads are in flight together
+  const bool isv = blockIdx.y != 0;  // K (0) or V (1); selected, not indexed, to keep the params out of local memory
+  const uint8_t* src = isv ? p.src[1] : p.src[0];
+  const float* scale = isv ? p.scale[1] : p.scale[0];
+  __nv_bfloat16* dst = isv ? p.dst[1] : p.dst[0];
   const int cpr = p.D / 16;  // 16-code chunks per (token, head) row
   const int per_batch = p.rows * p.H * cpr;
   const int total = p.B * per_batch;
-  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += gridDim.x * blockDim.x) {
-    const int b = idx / per_batch;
-    const int r = idx - b * per_batch;         // (token * H + h) * cpr + c within the batch entry
-    const int th = r / cpr, c = r - th * cpr;  // token-head row, chunk
-    const size_t row = static_cast<size_t>(b) * p.batch_rows * p.H + th;
-    const float sc = p.scale[which][row];
-    const uint4 u = *reinterpret_cast<const uint4*>(p.src[which] + row * p.D + c * 16);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-    uint32_t o[8];
+  const int stride = gridDim.x * blockDim.x;
+  for (int base = blockIdx.x * blockDim.x + threadIdx.x; base < total; base += U * stride) {
+    uint4 u[U];
+    float sc[U];
+    size_t row[U];
+    int c[U];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const __nv_fp8x2_storage_t q = static_cast<__nv_fp8x2_storage_t>((w[i] >> (16 * half)) & 0xFFFFu);
-        const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(q, __NV_E4M3);
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
-        o[2 * i + half] = pack_bf16(f.x * sc, f.y * sc);
+    for (int k = 0; k < U; ++k) {
+      const int idx = base + k * stride;
+      const int b = idx / per_batch;
+      const int r = idx - b * per_batch;  // (token * H + h) * cpr + c within the batch entry
+      const int th = r / cpr;             // token-head row
+      c[k] = r - th * cpr;
+      row[k] = static_cast<size_t>(b) * p.batch_rows * p.H + th;
+      sc[k] = 0.f;
+      u[k] = make_uint4(0u, 0u, 0u, 0u);
+      if (idx < total) {
+        sc[k] = scale[row[k]];
+        u[k] = *reinterpret_cast<const uint4*>(src + row[k] * p.D + c[k] * 16);
       }
     }
-    uint4* d = reinterpret_cast<uint4*>(p.dst[which] + row * p.D + c * 16);
-    d[0] = make_uint4(o[0], o[1], o[2], o[3]);
-    d[1] = make_uint4(o[4], o[5], o[6], o[7]);
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      if (base + k * stride >= total) continue;
+      const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+      uint32_t o[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const __nv_fp8x2_storage_t q = static_cast<__nv_fp8x2_storage_t>((w[i] >> (16 * half)) & 0xFFFFu);
+          const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(q, __NV_E4M3);
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+          o[2 * i + half] = pack_bf16(f.x * sc[k], f.y * sc[k]);
+        }
+      }
+      uint4* d = reinterpret_cast<uint4*>(dst + row[k] * p.D + c[k] * 16);
+      d[0] = make_uint4(o[0], o[1], o[2], o[3]);
+      d[1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
   }
 }
 
