@@ -143,6 +143,9 @@ ll_status ll_rope_apply(void* x, ll_dtype dtype, int B, int n_frames, int H, int
  * and "Short-Window Attention"). For an FP8 cache each (token, head) row is
  * stored as E4M3 codes of x / scale with scale = max|x| / 448 (1 for a zero
  * row), round-to-nearest-even with saturation.
+ * The library keeps no state: calling again with the same first_frame writes
+ * the same slots again (one call per denoising pass of the current frame, the
+ * last pass's K/V staying in the cache).
  * slots_out: optional HOST array of n_frames ints receiving the slots written.
  * Errors: LL_ERR_INVALID_ARG for NULL tensors, first_frame < 0,
  * n_frames < 1 or > n_local (a call may not overwrite its own frames),

@@ -44,12 +44,21 @@ class StreamOracle:
         t, r, c = token_positions(frame, self.grid_h, self.grid_w, self.t_offset)
         return rope_3d(x, t, r, c, self.omega, self.pairs)
 
-    def append(self, first_frame: int, k: np.ndarray, v: np.ndarray) -> None:
-        """Store frames first_frame.. (k, v: [F*N, H, D], K not yet rotated)."""
+    def append(self, first_frame: int, k: np.ndarray, v: np.ndarray, replace: bool = False) -> None:
+        """Store frames first_frame.. (k, v: [F*N, H, D], K not yet rotated).
+
+        replace=True re-writes the most recent frames instead (first_frame + F
+        - 1 == the last frame stored): one denoising pass of the current frame
+        or chunk (LongLive review, implementation table: several denoising
+        steps per frame) recomputes its K/V, and the next attention sees the
+        history plus this pass's K/V. The history itself is unchanged."""
         k = np.asarray(k, dtype=np.float64)
         v = np.asarray(v, dtype=np.float64)
         F = k.shape[0] // self.N
-        assert first_frame == self.last + 1, "frames must arrive in order"
+        if replace:
+            assert first_frame + F - 1 == self.last, "a pass re-writes the most recent frames"
+        else:
+            assert first_frame == self.last + 1, "frames must arrive in order"
         for fi in range(F):
             f = first_frame + fi
             sl = slice(fi * self.N, (fi + 1) * self.N)

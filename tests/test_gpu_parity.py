@@ -236,3 +236,25 @@ def test_attention_deterministic():
     outs = [swa.sink_window_attention(q, cache, 12, rope).clone() for _ in range(3)]
     torch.cuda.synchronize()
     assert all(torch.equal(outs[0], o) for o in outs[1:])
+
+
+@pytest.mark.parametrize("chunk", [False, True])
+def test_attention_denoising_passes(chunk):
+    """Several denoising passes per frame: each pass appends the frame's K/V
+    again (the library is stateless, so the frame's slot is simply
+    re-written) and attends; every pass is checked against the oracle stream
+    with the pass's K/V in place of the current frames'."""
+    w = W.replace(W.TINY, dtype="bf16", D=128, pairs=(22, 21, 21), name="tiny_passes", sigma_t=0.8, jitter_seed=3,
+                  query_frames=3 if chunk else 1, t_offset=700)
+    cache = swa.KVCache(1, w.H, w.D, w.N, "bf16")
+    rope = rope_of(w)
+    so = StreamOracle(w.H, w.D, w.grid_h, w.grid_w, omega_of(w), w.pairs, w.t_offset)
+    c = w.query_frames
+    for f0 in range(0, 15, c):
+        for ps in range(4):
+            q, k, v = W.qkv_frames(w, 10 * ps, f0, c)   # a different draw per pass
+            swa.kvcache_append(cache, k.cuda(), v.cuda(), f0, rope)
+            out = swa.sink_window_attention(q.cuda(), cache, f0, rope)
+            so.append(f0, np64(k[0]), np64(v[0]), replace=ps > 0)
+            ref = so.attend(np64(q[0]), f0)
+            assert_parity(np64(out[0]), ref, what=f"frame {f0} pass {ps}")

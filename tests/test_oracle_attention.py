@@ -106,3 +106,40 @@ def test_stream_rows_and_lse():
     part, lse_p = so.attend(q, 3, rows=[0, 5, 23], return_lse=True)
     assert np.allclose(part, full[[0, 5, 23]], atol=1e-14)
     assert np.allclose(lse_p, lse[:, [0, 5, 23]], atol=1e-14)
+
+
+@pytest.mark.parametrize("chunk", [1, 3])
+def test_stream_denoising_passes_match_dense_masked(chunk):
+    """Several denoising passes per frame (or chunk): each pass re-writes the
+    current frames' K/V (append(..., replace=True)) and attends. Every pass
+    equals one dense masked softmax over all frames in which the current
+    frames hold that pass's K/V and the earlier frames their last pass's."""
+    Wl = W.TINY
+    H, D, gh, gw = Wl.H, Wl.D, Wl.grid_h, Wl.grid_w
+    N = gh * gw
+    F, passes = 15, 3
+    om = rope.head_frequencies(H, Wl.pairs, 10000.0, 0.8, W.jitter_eps(6, H))
+    rng = np.random.default_rng(7)
+    Q = rng.standard_normal((passes, F * N, H, D))
+    K = rng.standard_normal((passes, F * N, H, D))
+    V = rng.standard_normal((passes, F * N, H, D))
+    Qr = [rope.rope_frames(Q[ps][None], 0, gh, gw, om, Wl.pairs, 40)[0] for ps in range(passes)]
+    Kr = [rope.rope_frames(K[ps][None], 0, gh, gw, om, Wl.pairs, 40)[0] for ps in range(passes)]
+    so = StreamOracle(H, D, gh, gw, om, Wl.pairs, t_offset=40)
+    kframe = np.repeat(np.arange(F), N)
+    for f0 in range(0, F, chunk):
+        cur = slice(f0 * N, (f0 + chunk) * N)
+        last = f0 + chunk - 1
+        A = set(window.attended_frames(last, 3, 9))
+        for ps in range(passes):
+            so.append(f0, K[ps][cur], V[ps][cur], replace=ps > 0)
+            got = so.attend(Q[ps][cur], f0)
+            kk = Kr[passes - 1].copy()
+            vv = V[passes - 1].copy()
+            kk[cur] = Kr[ps][cur]
+            vv[cur] = V[ps][cur]
+            ref = _dense_masked(Qr[ps][cur], kk, vv, np.repeat(np.arange(f0, f0 + chunk), N), kframe,
+                                lambda qf, kf: kf in A, 1 / np.sqrt(D))
+            assert np.allclose(got, ref, rtol=1e-11, atol=1e-11)
+    with pytest.raises(AssertionError):  # a pass may only re-write the most recent frames
+        so.append(0, K[0][:N], V[0][:N], replace=True)
