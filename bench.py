@@ -164,9 +164,10 @@ def max_over_ranks(value: float, dist: bool, device: str = "cuda") -> float:
 class Stream:
     """30 layers of caches and input pools on one GPU."""
 
-    def __init__(self, w: W.Workload, cache_dtype: str, device: str, seed_offset: int = 0):
+    def __init__(self, w: W.Workload, cache_dtype: str, device: str, seed_offset: int = 0, fused: bool = True):
         import sink_window_attention_b200 as swa
         self.swa = swa
+        self.fused = fused  # bf16 / f32 caches: ll_append_and_attend instead of append, then attention
         self.w = w
         self.device = device
         self.layers = w.layers
@@ -231,10 +232,16 @@ class Stream:
                     q, k, v = self.q[l][f % POOL], self.k[l][f % POOL], self.v[l][f % POOL]
                 else:
                     q, k, v = qkv(i, l)
-                swa.kvcache_append(self.caches[l], k, v, f, self.rope)
+                fused = self.fused and self.caches[l].dtype != "fp8"
+                if not fused:
+                    swa.kvcache_append(self.caches[l], k, v, f, self.rope)
+                    launches += 1
                 if attn_events is not None:
                     attn_events[0].record()
-                swa.sink_window_attention(q, self.caches[l], f, self.rope, out=self.out)
+                if fused:  # append + attention in one kernel
+                    swa.append_and_attend(self.caches[l], k, v, q, f, self.rope, out=self.out)
+                else:
+                    swa.sink_window_attention(q, self.caches[l], f, self.rope, out=self.out)
                 if self.caches[l].dtype == "fp8":
                     launches += 1  # the E4M3 -> bf16 staging kernel
                 if attn_events is not None:
@@ -242,7 +249,7 @@ class Stream:
                     attn_events[2].append((attn_events[0], attn_events[1]))
                     attn_events[0] = torch.cuda.Event(enable_timing=True)
                     attn_events[1] = torch.cuda.Event(enable_timing=True)
-                launches += 2
+                launches += 1
         return launches
 
 
@@ -253,7 +260,9 @@ def run_ours(args, rank, world, local_rank):
     import sink_window_attention_b200 as swa
     w = W.STREAM if args.cache == "bf16" else W.STREAM_FP8
     w = W.replace(w, layers=args.layers)
-    st = Stream(w, "bf16" if args.cache == "bf16" else "fp8", "cuda", seed_offset=replica_seed_offset(rank))
+    st = Stream(w, "bf16" if args.cache == "bf16" else "fp8", "cuda", seed_offset=replica_seed_offset(rank),
+                fused=not args.separate)
+    fused = st.fused and args.cache == "bf16"
     dist = world > 1
     if dist:
         import torch.distributed as tdist
@@ -317,7 +326,8 @@ def run_ours(args, rank, world, local_rank):
                    "recache": f"all {w.layers} layers at the segment start (X [{w.slots * w.N}, {w.dm}])",
                    "l2": "inputs larger than L2 (30 caches x 115 MB)", "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "tensor", "kernel": "sink_window_attention_kernel" + (
-                         " (+ E4M3 staging kernel inside the timed call)" if args.cache == "fp8" else ""),
+                         " (+ E4M3 staging kernel inside the timed call)" if args.cache == "fp8" else
+                         " (the frame's RoPE + append fused in: ll_append_and_attend)" if fused else ""),
                      "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_kind": f"{kind} bf16 dense, sustained",
@@ -384,8 +394,11 @@ def run_e2e(st: Stream, args, barrier, dist):
             f = SEGMENT * (s + 1) + i
             for l in range(L):
                 q, k, v = dev[b][l]
-                st.swa.kvcache_append(st.caches[l], k, v, f, st.rope)
-                st.swa.sink_window_attention(q, st.caches[l], f, st.rope, out=st.out)
+                if st.fused and st.caches[l].dtype != "fp8":
+                    st.swa.append_and_attend(st.caches[l], k, v, q, f, st.rope, out=st.out)
+                else:
+                    st.swa.kvcache_append(st.caches[l], k, v, f, st.rope)
+                    st.swa.sink_window_attention(q, st.caches[l], f, st.rope, out=st.out)
             free[b].record(comp)
             out_host[i].copy_(st.out, non_blocking=True)
 
@@ -630,6 +643,7 @@ def main():
     ap.add_argument("--cache", default="bf16", choices=["bf16", "fp8"])
     ap.add_argument("--layers", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--separate", action="store_true", help="append and attention as two calls (bf16 cache)")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--mode", default="stream", choices=["stream", "attention", "recache", "append"])
     ap.add_argument("--workload", default="wan", choices=["wan", "chunk"])

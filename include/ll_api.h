@@ -185,6 +185,33 @@ ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvc
                                    size_t workspace_bytes, void* stream);
 
 /*
+ * ll_kvcache_append of frames first_frame .. first_frame + n_frames - 1
+ * followed by ll_sink_window_attention of the same frames as queries, in one
+ * kernel: each CTA writes its share of the new frames' K/V into their slots
+ * while its first query tile loads, all CTAs meet at a grid-wide barrier, and
+ * only then is the cache read (LongLive review, "Frame Sink" and
+ * "Short-Window Attention": a new frame enters the window and attends to it).
+ * The results equal those of the two calls made one after the other.
+ * k, v, q, out: [B][n_frames*N][H][D] of `dtype`, which must be the cache's
+ * dtype (BF16 or F32; an FP8 cache needs the two separate calls). The other
+ * arguments are those of the two calls. workspace: device scratch of at least
+ * ll_append_and_attend_workspace_bytes(...) bytes, its contents need not be
+ * initialised (the grid barrier word is tagged with a per-launch generation,
+ * so it never needs resetting), and calls sharing it must be ordered.
+ * The launch is cooperative: every CTA must be resident at once, otherwise
+ * the launch fails with LL_ERR_CUDA instead of running.
+ * Errors: those of the two calls; LL_ERR_UNSUPPORTED for an FP8 cache or D
+ * other than 64 / 128 (bf16) and 64 (f32); LL_ERR_TIMEOUT (from
+ * ll_device_error) when the barrier wait gives up.
+ */
+size_t ll_append_and_attend_workspace_bytes(const ll_kvcache* cache, int n_frames);
+
+ll_status ll_append_and_attend(const ll_kvcache* cache, const void* k, const void* v, const void* q,
+                               ll_dtype dtype, long long first_frame, int n_frames,
+                               const ll_rope_desc* rope, float softmax_scale, void* out, float* lse,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Allocation-free variant of ll_sink_window_attention (the pages have no
  * counterpart; this is a library convenience).
  * Some callers cannot call cudaMalloc or any allocating routine: cudaMalloc

@@ -26,6 +26,7 @@ EXPORTED = (
     "ll_abi_version", "ll_last_error", "ll_slot_of_frame", "ll_device_error", "ll_rope_apply",
     "ll_kvcache_append", "ll_sink_window_attention_workspace_bytes", "ll_sink_window_attention",
     "ll_kv_recache_workspace_bytes", "ll_kv_recache", "ll_sink_window_attention_noalloc",
+    "ll_append_and_attend_workspace_bytes", "ll_append_and_attend",
 )
 NOALLOC_SCRATCH_BYTES = 48 * 1024 * 1024
 
@@ -75,8 +76,11 @@ def lib() -> ctypes.CDLL:
         L.ll_kv_recache_workspace_bytes.argtypes = [cp, i, i]
         L.ll_kv_recache_workspace_bytes.restype = sz
         L.ll_kv_recache.argtypes = [cp, vp, i, vp, vp, vp, f, ctypes.POINTER(ll_), i, rp, vp, sz, vp]
+        L.ll_append_and_attend_workspace_bytes.argtypes = [cp, i]
+        L.ll_append_and_attend_workspace_bytes.restype = sz
+        L.ll_append_and_attend.argtypes = [cp, vp, vp, vp, i, ll_, i, rp, f, vp, vp, vp, sz, vp]
         for name in EXPORTED[2:]:
-            if name not in ("ll_sink_window_attention_workspace_bytes", "ll_kv_recache_workspace_bytes"):
+            if not name.endswith("_workspace_bytes"):
                 getattr(L, name).restype = i
         _lib = L
     return _lib
@@ -202,10 +206,21 @@ def rope_apply(x: torch.Tensor, first_frame: int, rope: Rope, stream=None) -> to
     return x
 
 
+def _check_shape(cache: "KVCache", t: torch.Tensor, what: str) -> int:
+    """[B, F*N, H, D] on the cache's batch, heads and head dim; returns F."""
+    if t.dim() != 4 or t.shape[0] != cache.B or t.shape[2] != cache.H or t.shape[3] != cache.D or \
+            t.shape[1] % cache.N != 0 or not t.is_contiguous():
+        raise ValueError(f"{what} must be a contiguous [B={cache.B}, F*{cache.N}, {cache.H}, {cache.D}] tensor, "
+                         f"got {tuple(t.shape)}")
+    return t.shape[1] // cache.N
+
+
 def kvcache_append(cache: KVCache, k: torch.Tensor, v: torch.Tensor, first_frame: int,
                    rope: Optional[Rope], stream=None):
     """Write frames first_frame.. of k, v [B, F*N, H, D] into their slots; returns the slots."""
-    F = k.shape[1] // cache.N
+    F = _check_shape(cache, k, "k")
+    if _check_shape(cache, v, "v") != F:
+        raise ValueError("k and v must cover the same frames")
     slots = (ctypes.c_int * F)()
     _check(lib().ll_kvcache_append(ctypes.byref(cache.to_c()), _ptr(k), _ptr(v), _dtype_code(k.dtype), first_frame,
                                    F, _rope_ref(rope), slots, _stream(stream)))
@@ -236,7 +251,7 @@ def sink_window_attention(q: torch.Tensor, cache: KVCache, first_frame: int, rop
                           lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                           stream=None) -> torch.Tensor:
     """Attention of query frames first_frame.. (q [B, F*N, H, D]) over the cache."""
-    F = q.shape[1] // cache.N
+    F = _check_shape(cache, q, "q")
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:
@@ -248,12 +263,36 @@ def sink_window_attention(q: torch.Tensor, cache: KVCache, first_frame: int, rop
     return out
 
 
+def append_and_attend_workspace_bytes(cache: KVCache, n_frames: int) -> int:
+    return int(lib().ll_append_and_attend_workspace_bytes(ctypes.byref(cache.to_c()), n_frames))
+
+
+def append_and_attend(cache: KVCache, k: torch.Tensor, v: torch.Tensor, q: torch.Tensor, first_frame: int,
+                      rope: Optional[Rope], softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                      lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """ll_append_and_attend: append frames first_frame.. (k, v [B, F*N, H, D])
+    and attend with their queries q in one kernel (BF16 / F32 caches)."""
+    F = _check_shape(cache, q, "q")
+    if _check_shape(cache, k, "k") != F or _check_shape(cache, v, "v") != F:
+        raise ValueError("k, v and q must cover the same frames")
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = workspace_for(append_and_attend_workspace_bytes(cache, F), q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().ll_append_and_attend(ctypes.byref(cache.to_c()), _ptr(k), _ptr(v), _ptr(q), _dtype_code(q.dtype),
+                                      first_frame, F, _rope_ref(rope), float(softmax_scale), _ptr(out), _ptr(lse),
+                                      _ptr(workspace), ws_bytes, _stream(stream)))
+    return out
+
+
 def sink_window_attention_noalloc(q: torch.Tensor, cache: KVCache, first_frame: int, rope: Optional[Rope],
                                   softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
                                   lse: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """ll_sink_window_attention_noalloc: the same attention with the library's
     static scratch array instead of a caller workspace (allocates nothing)."""
-    F = q.shape[1] // cache.N
+    F = _check_shape(cache, q, "q")
     if out is None:
         out = torch.empty_like(q)
     _check(lib().ll_sink_window_attention_noalloc(_ptr(q), _dtype_code(q.dtype), ctypes.byref(cache.to_c()),

@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <string>
 
@@ -164,7 +165,7 @@ size_t attention_workspace(int units) {
 
 template <class TR>
 ll_status launch_attention(ll::AttnParams p, const ll_kvcache* c, long long S, void* workspace, size_t ws_bytes,
-                           cudaStream_t stream) {
+                           cudaStream_t stream, bool cooperative = false) {
   p.q_tiles = (p.Tq + TR::BM - 1) / TR::BM;
   p.nkv = (p.Nk + TR::BN - 1) / TR::BN;
   p.units = p.q_tiles * c->H * c->B;
@@ -195,8 +196,34 @@ ll_status launch_attention(ll::AttnParams p, const ll_kvcache* c, long long S, v
   }
   if (cudaMemsetAsync(p.counters, 0, p.units * sizeof(int), stream) != cudaSuccess)
     return check_launch("cudaMemsetAsync(attention counters)");
-  kern<<<p.grid, TR::THREADS, TR::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
-  return check_launch("sink_window_attention_kernel");
+  if (!cooperative) {
+    kern<<<p.grid, TR::THREADS, TR::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
+    return check_launch("sink_window_attention_kernel");
+  }
+  // fused append: the CTAs meet at a grid barrier, so they must all be
+  // resident at once (the launch fails instead of running otherwise)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.grid, 1, 1);
+  cfg.blockDim = dim3(TR::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = TR::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tmQ, tmK, tmV, p) != cudaSuccess)
+    return check_launch("sink_window_attention_kernel (cooperative, fused append)");
+  return check_launch("sink_window_attention_kernel (cooperative, fused append)");
+}
+
+// Launch generation of the fused append's grid barrier word (never 0, so a
+// zero-filled word never matches).
+unsigned int next_generation() {
+  static std::atomic<unsigned int> gen{0};
+  unsigned int g = ++gen;
+  if (g == 0) g = ++gen;
+  return g;
 }
 
 // Bytes of the bf16 copy of an FP8 cache that attention over an FP8 cache
@@ -410,6 +437,91 @@ ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvc
   if (f32 && cache->D == 64)
     return launch_attention<ll::AttnTraits<64, float>>(p, cache, S, workspace, workspace_bytes, s);
   return fail(LL_ERR_UNSUPPORTED, "attention supports D = 64 or 128 (bf16) and D = 64 (f32); got D = %d", cache->D);
+}
+
+size_t ll_append_and_attend_workspace_bytes(const ll_kvcache* cache, int n_frames) {
+  if (cache == nullptr || n_frames < 1 || cache->tokens_per_frame < 1 || cache->H < 1 || cache->B < 1 ||
+      cache->dtype == LL_FP8_E4M3)
+    return 0;
+  return attention_scratch_bytes(cache, n_frames) + 256;  // + the grid barrier word
+}
+
+ll_status ll_append_and_attend(const ll_kvcache* cache, const void* k, const void* v, const void* q, ll_dtype dtype,
+                               long long first_frame, int n_frames, const ll_rope_desc* rope, float softmax_scale,
+                               void* out, float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  g_last_error.clear();
+  ll_status st = check_cache(cache);
+  if (st != LL_OK) return st;
+  if (cache->dtype == LL_FP8_E4M3)
+    return fail(LL_ERR_UNSUPPORTED, "the fused append + attention takes a BF16 or F32 cache (FP8: call "
+                                    "ll_kvcache_append, then ll_sink_window_attention)");
+  if (dtype != cache->dtype) return fail(LL_ERR_INVALID_ARG, "k, v and q must have the cache's dtype");
+  if (k == nullptr || v == nullptr || q == nullptr || out == nullptr)
+    return fail(LL_ERR_INVALID_ARG, "k, v, q and out must be non-NULL");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(q) || !aligned16(out))
+    return fail(LL_ERR_INVALID_ARG, "k, v, q and out must be 16-byte aligned");
+  if (first_frame < 0) return fail(LL_ERR_INVALID_ARG, "first_frame must be >= 0");
+  if (n_frames < 1 || n_frames > cache->n_local)
+    return fail(LL_ERR_INVALID_ARG, "n_frames = %d must lie in [1, n_local = %d]", n_frames, cache->n_local);
+  if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale))
+    return fail(LL_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  const size_t need = ll_append_and_attend_workspace_bytes(cache, n_frames);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(LL_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu required", workspace_bytes, need);
+  if (!aligned16(workspace)) return fail(LL_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  if ((st = check_grid(rope, cache->tokens_per_frame)) != LL_OK) return st;
+  const bool f32 = cache->dtype == LL_F32;
+  if (!((!f32 && (cache->D == 128 || cache->D == 64)) || (f32 && cache->D == 64)))
+    return fail(LL_ERR_UNSUPPORTED, "attention supports D = 64 or 128 (bf16) and D = 64 (f32); got D = %d", cache->D);
+  // the append part, exactly as ll_kvcache_append sets it up
+  ll::AttnParams p{};
+  ll::AppendParams& ap = p.ap;
+  if ((st = make_rope(rope, cache->H, cache->D, first_frame, &ap.rp)) != LL_OK) return st;
+  ap.k_in = k;
+  ap.v_in = v;
+  ap.k_cache = cache->k;
+  ap.v_cache = cache->v;
+  ap.B = cache->B;
+  ap.F = n_frames;
+  ap.N = cache->tokens_per_frame;
+  ap.H = cache->H;
+  ap.D = cache->D;
+  ap.n_sink = cache->n_sink;
+  ap.n_local = cache->n_local;
+  ap.first_frame = first_frame;
+  if (ll::append_items(ap) >= (1LL << 31))
+    return fail(LL_ERR_UNSUPPORTED, "tensor too large for one call (%lld items)", ll::append_items(ap));
+  // the append's frequency tables are built in the kernel's K stages
+  const size_t tables = ll::append_smem_bytes(n_frames, cache->H, cache->D, ap.rp.pt);
+  const size_t kstages = cache->D == 128 ? ll::AttnTraits<128, __nv_bfloat16>::KST * ll::AttnTraits<128, __nv_bfloat16>::KV_BYTES
+                                         : (f32 ? ll::AttnTraits<64, float>::KST * ll::AttnTraits<64, float>::KV_BYTES
+                                                : ll::AttnTraits<64, __nv_bfloat16>::KST * ll::AttnTraits<64, __nv_bfloat16>::KV_BYTES);
+  if (tables > kstages)
+    return fail(LL_ERR_UNSUPPORTED, "frequency tables of %zu bytes exceed %zu", tables, kstages);
+  // the attention part, exactly as ll_sink_window_attention sets it up
+  const long long S = cache->n_sink + cache->n_local;
+  const long long last = first_frame + n_frames - 1;
+  const long long valid_slots = last + 1 < S ? last + 1 : S;
+  if ((st = make_rope(rope, cache->H, cache->D, first_frame, &p.rp)) != LL_OK) return st;
+  p.q = q;
+  p.out = out;
+  p.lse = lse;
+  p.B = cache->B;
+  p.H = cache->H;
+  p.Tq = n_frames * cache->tokens_per_frame;
+  p.Nk = static_cast<int>(valid_slots * cache->tokens_per_frame);
+  p.softmax_scale = softmax_scale;
+  p.N = cache->tokens_per_frame;
+  p.fuse_append = 1;
+  p.gen = next_generation();
+  p.grid_bar = reinterpret_cast<unsigned long long*>(static_cast<char*>(workspace) +
+                                                     attention_scratch_bytes(cache, n_frames));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!f32 && cache->D == 128)
+    return launch_attention<ll::AttnTraits<128, __nv_bfloat16>>(p, cache, S, workspace, workspace_bytes, s, true);
+  if (!f32)
+    return launch_attention<ll::AttnTraits<64, __nv_bfloat16>>(p, cache, S, workspace, workspace_bytes, s, true);
+  return launch_attention<ll::AttnTraits<64, float>>(p, cache, S, workspace, workspace_bytes, s, true);
 }
 
 }  // extern "C"

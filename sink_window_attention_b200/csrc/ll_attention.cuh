@@ -98,6 +98,13 @@ struct AttnParams {
   long long total;   // units * nkv
   int* counters;     // [units] arrivals per unit (zeroed by the host before the launch)
   float* partials;   // [(grid + units) * SLOT_FLOATS]
+  // Fused append (ll_append_and_attend): every CTA first writes its share of
+  // the new frames' K/V into the cache, then all CTAs meet at a grid barrier
+  // (cooperative launch: all CTAs are co-resident) before any K/V is read.
+  int fuse_append;
+  unsigned int gen;                // generation tag of this launch in the barrier word
+  unsigned long long* grid_bar;    // [generation:32 | arrivals:32]
+  AppendParams ap;                 // the append (input dtype = cache dtype = T)
 };
 
 // A piece: key tiles [j0, j0 + n) of unit u.
@@ -255,14 +262,38 @@ __global__ void __launch_bounds__(384, 1)
 
   // The first piece's Q tile comes in by TMA; warps 2-11 rotate it together
   // (the softmax warpgroups have nothing to do before it). Later pieces:
-  // warps 2-3.
+  // warps 2-3. With a fused append, the whole CTA first writes its share of
+  // the new frames into the cache while that Q copy is in flight.
   {
     long long it0 = it_begin;
     Piece pc0;
     next_piece(it0, pc0);
+    if (threadIdx.x == 64) tma_q_tile<TR>(sQ, &tmQ, &q_tma[0], p, pc0.u);
+    if (p.fuse_append) {
+      // the append's tables live in the K stages, which TMA fills only after the barrier
+      float* s_aom = reinterpret_cast<float*>(sK);
+      float* s_atc = s_aom + p.ap.H * (p.ap.D / 2);
+      if (p.ap.rp.enabled) build_append_tables(s_aom, s_atc, p.ap);
+      const long long items = append_items(p.ap);
+      const long long b0 = g * items / p.grid, b1 = (g + 1) * items / p.grid;
+      for (long long i = b0 + threadIdx.x; i < b1; i += blockDim.x) {
+        const AppendItem ai = append_item(p.ap, static_cast<int>(i));
+        float kx[kAppendMaxHg][8], vx[kAppendMaxHg][8];
+        append_load<T>(p.ap, ai, true, kx, vx);
+        if (p.ap.rp.enabled) append_rotate(p.ap, ai, s_aom, s_atc, kx);
+        append_store_plain<T>(p.ap, ai, kx, vx);
+      }
+      // the cache rows written here are read by TMA (async proxy) after the
+      // barrier, and TMA refills the K stages that held the tables
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      fence_proxy_async_smem();
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x == 0) grid_barrier(p.grid_bar, p.gen, static_cast<unsigned int>(p.grid), s_abort);
+      __syncthreads();
+    }
     if (warp >= 2) {
       const int tid = threadIdx.x - 64;  // 0..319
-      if (tid == 0) tma_q_tile<TR>(sQ, &tmQ, &q_tma[0], p, pc0.u);
       if (p.rp.enabled)
         for (int j = tid; j < D / 2; j += 320) s_omega[j] = omega_of(p.rp, (pc0.u / p.q_tiles) % p.H, j);
       asm volatile("bar.sync 4, 320;" ::: "memory");
@@ -282,6 +313,7 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
+      if (p.fuse_append) asm volatile("fence.proxy.async.global;" ::: "memory");  // see the append above
       // K and V walk the same tile sequence with cursors of their own; each
       // is loaded as soon as its ring has a free stage, so K runs ahead of V
       // by as many tiles as its ring holds

@@ -103,6 +103,44 @@ __device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, v
   }
 }
 
+// Grid-wide barrier of `count` co-resident CTAs (one thread per CTA calls it).
+// The 64-bit word holds [generation:32 | arrivals:32]; a word left by an older
+// launch (another generation) counts as no arrivals, so it never needs
+// resetting. The first CTA to arrive retags a stale word with this launch's
+// generation (the only compare-and-swap: CTAs that lose that race see the new
+// tag in the value it returns); every CTA then arrives with one atomic add, so
+// arrivals do not serialise on retried swaps. Bounded like every wait: on
+// timeout it records kErrWaitTimeout, sets *abort and returns false.
+__device__ __forceinline__ bool grid_barrier(unsigned long long* word, unsigned int gen, unsigned int count,
+                                             volatile int* abort) {
+  unsigned long long cur;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(cur) : "l"(word) : "memory");
+  for (int guard = 0; static_cast<unsigned int>(cur >> 32) != gen; ++guard) {
+    const unsigned long long prev = atomicCAS(word, cur, static_cast<unsigned long long>(gen) << 32);
+    if (prev == cur) break;
+    cur = prev;
+    if (guard > 64) {
+      atomicOr(&g_error_word, kErrWaitTimeout);
+      *abort = 1;
+      return false;
+    }
+  }
+  atomicAdd(word, 1ull);
+  const long long t0 = clock64();
+  while (true) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(word) : "memory");
+    if (static_cast<unsigned int>(v >> 32) == gen && static_cast<unsigned int>(v) >= count) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitLimitCycles) {
+      atomicOr(&g_error_word, kErrWaitTimeout);
+      *abort = 1;
+      return false;
+    }
+    __nanosleep(64);
+  }
+}
+
 // Bounded wait used during teardown after an abort: ignores the abort flag.
 __device__ __forceinline__ bool mbar_wait_teardown(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_addr(bar);

@@ -222,110 +222,155 @@ __host__ __device__ __forceinline__ size_t append_smem_bytes(int F, int H, int D
   return (static_cast<size_t>(H) * (D / 2) + 2 * static_cast<size_t>(F) * H * pt) * sizeof(float);
 }
 
+// Frequency table [H][D/2] and the temporal band's cos/sin [F][H][pt][2] in
+// shared memory, built by the whole block (two block barriers).
+__device__ __forceinline__ void build_append_tables(float* s_omega, float* s_tcs, const AppendParams& p) {
+  const int P = p.D / 2;
+  build_omega(s_omega, p.rp, 0, p.H, P);
+  __syncthreads();
+  const int nt = p.F * p.H * p.rp.pt;
+  for (int idx = threadIdx.x; idx < nt; idx += blockDim.x) {
+    const int f = idx / (p.H * p.rp.pt), rem = idx - f * (p.H * p.rp.pt);
+    const int h = rem / p.rp.pt, j = rem - h * p.rp.pt;
+    float sn, cs;
+    sincos_reduced(static_cast<float>(p.rp.t_first + f) * s_omega[h * P + j], sn, cs);
+    s_tcs[2 * idx] = cs;
+    s_tcs[2 * idx + 1] = sn;
+  }
+  __syncthreads();
+}
+
+// Number of append work items: (token, 8-element chunk position, group of
+// append_heads_per_thread(H) heads).
+__host__ __device__ __forceinline__ long long append_items(const AppendParams& p) {
+  return static_cast<long long>(p.B) * p.F * p.N * (p.D / 8) * (p.H / append_heads_per_thread(p.H));
+}
+
+// One work item: where its chunks come from and go to.
+struct AppendItem {
+  int c, h0, fi, n;
+  size_t src0, dst0;  // element offsets of the group's first head in the input and in the cache
+};
+
+__device__ __forceinline__ AppendItem append_item(const AppendParams& p, int i) {
+  const int cpr = p.D / 8;
+  const int hg = append_heads_per_thread(p.H);
+  const int ngroups = p.H / hg;
+  AppendItem it;
+  const int grow = i / cpr;  // (b * F*N + tok) * ngroups + group
+  it.c = i - grow * cpr;
+  const int bt = grow / ngroups;
+  it.h0 = (grow - bt * ngroups) * hg;
+  const int FN = p.F * p.N;
+  const int b = bt / FN;
+  const int tok = bt - b * FN;
+  it.fi = tok / p.N;
+  it.n = tok - it.fi * p.N;
+  const int S = p.n_sink + p.n_local;
+  const int slot = cache_slot(p.first_frame + it.fi, p.n_sink, p.n_local);
+  it.src0 = (static_cast<size_t>(bt) * p.H + it.h0) * p.D + it.c * 8;
+  it.dst0 = ((static_cast<size_t>(b) * S * p.N + static_cast<size_t>(slot) * p.N + it.n) * p.H + it.h0) * p.D +
+            it.c * 8;
+  return it;
+}
+
+template <typename Tin>
+__device__ __forceinline__ void append_load(const AppendParams& p, const AppendItem& it, bool active,
+                                            float (&kx)[kAppendMaxHg][8], float (&vx)[kAppendMaxHg][8]) {
+  const int hg = append_heads_per_thread(p.H);
+  const Tin* kin = static_cast<const Tin*>(p.k_in);
+  const Tin* vin = static_cast<const Tin*>(p.v_in);
+#pragma unroll
+  for (int k = 0; k < kAppendMaxHg; ++k) {
+    if (active && k < hg) {
+      load_chunk8<Tin>(kin + it.src0 + static_cast<size_t>(k) * p.D, kx[k]);
+      load_chunk8<Tin>(vin + it.src0 + static_cast<size_t>(k) * p.D, vx[k]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) kx[k][e] = vx[k][e] = 0.f;
+    }
+  }
+}
+
+// Rotate the K chunks of an item: a row- or column-band pair has one angle for
+// all heads; a temporal-band pair takes its head's cos/sin from the table.
+__device__ __forceinline__ void append_rotate(const AppendParams& p, const AppendItem& it, const float* s_omega,
+                                              const float* s_tcs, float (&kx)[kAppendMaxHg][8]) {
+  const int hg = append_heads_per_thread(p.H);
+  const int pth = p.rp.pt + p.rp.ph;
+  const float pos_r = static_cast<float>(it.n / p.rp.grid_w), pos_c = static_cast<float>(it.n % p.rp.grid_w);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int j = it.c * 4 + q;
+    float cs[kAppendMaxHg], sn[kAppendMaxHg];
+    if (j < p.rp.pt) {
+#pragma unroll
+      for (int k = 0; k < kAppendMaxHg; ++k) {
+        const int e = k < hg ? ((it.fi * p.H + it.h0 + k) * p.rp.pt + j) : 0;
+        cs[k] = s_tcs[2 * e];
+        sn[k] = s_tcs[2 * e + 1];
+      }
+    } else {
+      float s1, c1;
+      sincos_reduced((j < pth ? pos_r : pos_c) * s_omega[j], s1, c1);
+#pragma unroll
+      for (int k = 0; k < kAppendMaxHg; ++k) {
+        cs[k] = c1;
+        sn[k] = s1;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kAppendMaxHg; ++k) {
+      const float x0 = kx[k][2 * q], x1 = kx[k][2 * q + 1];
+      kx[k][2 * q] = x0 * cs[k] - x1 * sn[k];
+      kx[k][2 * q + 1] = x0 * sn[k] + x1 * cs[k];
+    }
+  }
+}
+
+template <typename C>
+__device__ __forceinline__ void append_store_plain(const AppendParams& p, const AppendItem& it,
+                                                   const float (&kx)[kAppendMaxHg][8],
+                                                   const float (&vx)[kAppendMaxHg][8]) {
+  const int hg = append_heads_per_thread(p.H);
+#pragma unroll
+  for (int k = 0; k < kAppendMaxHg; ++k)
+    if (k < hg) {
+      store_chunk8<C>(static_cast<C*>(p.k_cache) + it.dst0 + static_cast<size_t>(k) * p.D, kx[k]);
+      store_chunk8<C>(static_cast<C*>(p.v_cache) + it.dst0 + static_cast<size_t>(k) * p.D, vx[k]);
+    }
+}
+
 template <typename Tin, typename C>
 __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
   extern __shared__ float s_tab[];      // omega [H][D/2], then cos, sin of the temporal band [F][H][pt][2]
-  const int P = p.D / 2;
   float* s_omega = s_tab;
-  float* s_tcs = s_tab + p.H * P;
+  float* s_tcs = s_tab + p.H * (p.D / 2);
   const int cpr = p.D / 8;                        // chunks per (token, head) row
   const int hg = append_heads_per_thread(p.H);    // heads per thread
-  const int ngroups = p.H / hg;
-  const int total = p.B * p.F * p.N * ngroups * cpr;  // < 2^31, checked on the host
-  const int FN = p.F * p.N;
-  const int S = p.n_sink + p.n_local;
-  const int pth = p.rp.pt + p.rp.ph;
-  const Tin* kin = static_cast<const Tin*>(p.k_in);
-  const Tin* vin = static_cast<const Tin*>(p.v_in);
+  const int total = static_cast<int>(append_items(p));  // < 2^31, checked on the host
   const int stride = gridDim.x * blockDim.x;
   float kx[kAppendMaxHg][8], vx[kAppendMaxHg][8];
-  auto load = [&](int idx) {
-    const bool active = idx < total;
-    const int i = active ? idx : 0;
-    const int grow = i / cpr, c = i - grow * cpr;
-    const int bt = grow / ngroups;
-    const size_t src0 = (static_cast<size_t>(bt) * p.H + (grow - bt * ngroups) * hg) * p.D + c * 8;
-#pragma unroll
-    for (int k = 0; k < kAppendMaxHg; ++k) {
-      if (active && k < hg) {
-        load_chunk8<Tin>(kin + src0 + static_cast<size_t>(k) * p.D, kx[k]);
-        load_chunk8<Tin>(vin + src0 + static_cast<size_t>(k) * p.D, vx[k]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) kx[k][e] = vx[k][e] = 0.f;
-      }
-    }
-  };
   // the first chunks' loads go out before the tables are built, so the
   // table work overlaps their latency
   int base = blockIdx.x * blockDim.x;
-  load(base + threadIdx.x);
-  if (p.rp.enabled) {
-    build_omega(s_omega, p.rp, 0, p.H, P);
-    __syncthreads();
-    const int nt = p.F * p.H * p.rp.pt;
-    for (int idx = threadIdx.x; idx < nt; idx += blockDim.x) {
-      const int f = idx / (p.H * p.rp.pt), rem = idx - f * (p.H * p.rp.pt);
-      const int h = rem / p.rp.pt, j = rem - h * p.rp.pt;
-      float sn, cs;
-      sincos_reduced(static_cast<float>(p.rp.t_first + f) * s_omega[h * P + j], sn, cs);
-      s_tcs[2 * idx] = cs;
-      s_tcs[2 * idx + 1] = sn;
-    }
+  {
+    const int idx = base + threadIdx.x;
+    append_load<Tin>(p, append_item(p, idx < total ? idx : 0), idx < total, kx, vx);
   }
-  __syncthreads();
+  if (p.rp.enabled) build_append_tables(s_omega, s_tcs, p);
   // All threads of the block run the same number of iterations, so the
   // shuffles of the FP8 path always see full warps.
   for (; base < total; base += stride) {
     const int idx = base + threadIdx.x;
     const bool active = idx < total;
-    const int i = active ? idx : 0;
-    const int grow = i / cpr;                     // (b * F*N + tok) * ngroups + group
-    const int c = i - grow * cpr;
-    const int bt = grow / ngroups;
-    const int h0 = (grow - bt * ngroups) * hg;
-    const int b = bt / FN;
-    const int tok = bt - b * FN;
-    const int fi = tok / p.N;
-    const int n = tok - fi * p.N;
-    const int slot = cache_slot(p.first_frame + fi, p.n_sink, p.n_local);
-    const size_t dst0 = ((static_cast<size_t>(b) * S * p.N + static_cast<size_t>(slot) * p.N + n) * p.H + h0) * p.D +
-                        c * 8;
-    if (active && p.rp.enabled) {
-      const float pos_r = static_cast<float>(n / p.rp.grid_w), pos_c = static_cast<float>(n % p.rp.grid_w);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int j = c * 4 + q;
-        float cs[kAppendMaxHg], sn[kAppendMaxHg];
-        if (j < p.rp.pt) {  // temporal band: per-head angle from the table
-#pragma unroll
-          for (int k = 0; k < kAppendMaxHg; ++k) {
-            const int e = k < hg ? ((fi * p.H + h0 + k) * p.rp.pt + j) : 0;
-            cs[k] = s_tcs[2 * e];
-            sn[k] = s_tcs[2 * e + 1];
-          }
-        } else {  // row / column band: one angle for all heads
-          float s1, c1;
-          sincos_reduced((j < pth ? pos_r : pos_c) * s_omega[j], s1, c1);
-#pragma unroll
-          for (int k = 0; k < kAppendMaxHg; ++k) {
-            cs[k] = c1;
-            sn[k] = s1;
-          }
-        }
-#pragma unroll
-        for (int k = 0; k < kAppendMaxHg; ++k) {
-          const float x0 = kx[k][2 * q], x1 = kx[k][2 * q + 1];
-          kx[k][2 * q] = x0 * cs[k] - x1 * sn[k];
-          kx[k][2 * q + 1] = x0 * sn[k] + x1 * cs[k];
-        }
-      }
-    }
+    const AppendItem it = append_item(p, active ? idx : 0);
+    if (active && p.rp.enabled) append_rotate(p, it, s_omega, s_tcs, kx);
     if constexpr (sizeof(C) == 1) {
       // per (token, head) row: scale = max|x| / 448 over the row's D values,
       // which lie in the cpr consecutive lanes of this chunk position's group
-      uint8_t* kc = static_cast<uint8_t*>(p.k_cache) + dst0;
-      uint8_t* vc = static_cast<uint8_t*>(p.v_cache) + dst0;
+      uint8_t* kc = static_cast<uint8_t*>(p.k_cache) + it.dst0;
+      uint8_t* vc = static_cast<uint8_t*>(p.v_cache) + it.dst0;
 #pragma unroll
       for (int k = 0; k < kAppendMaxHg; ++k) {
         if (k >= hg) break;  // hg is uniform across the grid
@@ -344,24 +389,20 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
         if (active) {
           *reinterpret_cast<uint2*>(kc + static_cast<size_t>(k) * p.D) = encode_chunk8_e4m3(kx[k], ks);
           *reinterpret_cast<uint2*>(vc + static_cast<size_t>(k) * p.D) = encode_chunk8_e4m3(vx[k], vs);
-          if (c == 0) {
-            const size_t srow = dst0 / p.D + k;
+          if (it.c == 0) {
+            const size_t srow = it.dst0 / p.D + k;
             p.k_scale[srow] = ks;
             p.v_scale[srow] = vs;
           }
         }
       }
     } else {
-      if (active) {
-#pragma unroll
-        for (int k = 0; k < kAppendMaxHg; ++k)
-          if (k < hg) {
-            store_chunk8<C>(static_cast<C*>(p.k_cache) + dst0 + static_cast<size_t>(k) * p.D, kx[k]);
-            store_chunk8<C>(static_cast<C*>(p.v_cache) + dst0 + static_cast<size_t>(k) * p.D, vx[k]);
-          }
-      }
+      if (active) append_store_plain<C>(p, it, kx, vx);
     }
-    if (base + stride < total) load(base + stride + threadIdx.x);  // uniform condition
+    if (base + stride < total) {  // uniform condition
+      const int nidx = base + stride + threadIdx.x;
+      append_load<Tin>(p, append_item(p, nidx < total ? nidx : 0), nidx < total, kx, vx);
+    }
   }
 }
 

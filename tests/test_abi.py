@@ -128,3 +128,35 @@ def test_recache_validation(L):
     assert call(dm=100) == swa.LL_ERR_UNSUPPORTED
     assert call(cache=_cache(H=3)) == swa.LL_ERR_UNSUPPORTED        # H*D = 384 is not a multiple of 256
     assert call(cache=_cache(dtype=swa.LL_F32)) == swa.LL_ERR_UNSUPPORTED
+
+
+def _fused(L, cache, rope=None, first=0, nf=1, scale=0.0, ws=1 << 24, ws_bytes=1 << 30, k=1 << 20, v=1 << 21,
+           q=1 << 22, out=1 << 23, dt=swa.LL_BF16):
+    return L.ll_append_and_attend(ctypes.byref(cache), k, v, q, dt, first, nf,
+                                  ctypes.byref(rope) if rope is not None else None, scale, out, None, ws,
+                                  ws_bytes, None)
+
+
+def test_fused_append_attention_validation(L):
+    """Every malformed call is rejected on the host, before any launch."""
+    fp8 = _cache(dtype=swa.LL_FP8_E4M3, k_scale=1 << 25, v_scale=1 << 26)
+    assert L.ll_append_and_attend_workspace_bytes(ctypes.byref(fp8), 1) == 0
+    assert _fused(L, fp8) == swa.LL_ERR_UNSUPPORTED                 # FP8: the two separate calls
+    assert _fused(L, _cache(D=96)) == swa.LL_ERR_UNSUPPORTED        # no kernel for D = 96
+    need = L.ll_append_and_attend_workspace_bytes(ctypes.byref(_cache()), 1)
+    assert need > L.ll_sink_window_attention_workspace_bytes(ctypes.byref(_cache()), 1)  # + the barrier word
+    bad = [
+        dict(cache=_cache(), dt=swa.LL_F32),                         # not the cache's dtype
+        dict(cache=_cache(), k=None),
+        dict(cache=_cache(), q=(1 << 22) + 4),                       # misaligned
+        dict(cache=_cache(), first=-1),
+        dict(cache=_cache(), nf=0),
+        dict(cache=_cache(), nf=10),
+        dict(cache=_cache(), scale=float("nan")),
+        dict(cache=_cache(), ws_bytes=need - 1),
+        dict(cache=_cache(), rope=_rope(grid_h=29)),
+    ]
+    for kw in bad:
+        st = _fused(L, **kw)
+        assert st == swa.LL_ERR_INVALID_ARG, (kw, st)
+        assert swa.last_error() != ""

@@ -258,3 +258,41 @@ def test_attention_denoising_passes(chunk):
             so.append(f0, np64(k[0]), np64(v[0]), replace=ps > 0)
             ref = so.attend(np64(q[0]), f0)
             assert_parity(np64(out[0]), ref, what=f"frame {f0} pass {ps}")
+
+
+@pytest.mark.parametrize("name", ["wan", "chunk", "tiny", "tiny_d64_b2"])
+def test_fused_append_attention_matches_separate_calls(name):
+    """ll_append_and_attend gives bit-identical outputs, LSE and cache contents
+    to ll_kvcache_append followed by ll_sink_window_attention, from the first
+    frame through the ring wrap."""
+    w = {"wan": W.WAN, "chunk": W.CHUNK, "tiny": W.TINY,
+         "tiny_d64_b2": W.replace(W.TINY, dtype="bf16", name="tiny_d64_b2", B=2)}[name]
+    rope = rope_of(w)
+    c = w.query_frames
+    caches = [swa.KVCache(w.B, w.H, w.D, w.N, w.dtype) for _ in range(2)]
+    frames = range(0, 15, c) if w.N < 100 else [0, 3 * c, 11, 12 * c] if c == 1 else [0, 3, 9, 12]
+    for f0 in frames:
+        q, k, v = (t.cuda() for t in W.qkv_frames(w, 0, f0, c))   # [w.B, c*N, H, D]
+        lse = [torch.empty(w.B, w.H, q.shape[1], device="cuda", dtype=torch.float32) for _ in range(2)]
+        swa.kvcache_append(caches[0], k, v, f0, rope)
+        o0 = swa.sink_window_attention(q, caches[0], f0, rope, lse=lse[0])
+        o1 = swa.append_and_attend(caches[1], k, v, q, f0, rope, lse=lse[1])
+        torch.cuda.synchronize()
+        assert torch.equal(o0, o1), f"frame {f0}"
+        assert torch.equal(lse[0], lse[1]), f"frame {f0}"
+        assert torch.equal(caches[0].k, caches[1].k) and torch.equal(caches[0].v, caches[1].v), f"frame {f0}"
+
+
+def test_fused_append_attention_stream_parity():
+    """The fused call against the oracle stream: chunks with jitter."""
+    w = W.CHUNK
+    cache = swa.KVCache(w.B, w.H, w.D, w.N, w.dtype)
+    rope = rope_of(w)
+    so = StreamOracle(w.H, w.D, w.grid_h, w.grid_w, omega_of(w), w.pairs, w.t_offset)
+    for f0 in range(0, 18, 3):
+        q, k, v = W.qkv_frames(w, 0, f0, 3)
+        out = swa.append_and_attend(cache, k.cuda(), v.cuda(), q.cuda(), f0, rope)
+        so.append(f0, np64(k[0]), np64(v[0]))
+        rows = sample_rows(q.shape[1], 24, f0)
+        ref = so.attend(np64(q[0]), f0, rows=rows)
+        assert_parity(np64(out[0])[rows], ref, what=f"fused chunk {f0}")
