@@ -76,7 +76,9 @@ struct AttnTraits {
   // that ptxas allocated exactly LAUNCH_REGS.
   static constexpr int LAUNCH_REGS = 168, REGS_LOW = 72, REGS_HIGH = 216;
   static_assert(128 * REGS_LOW + 256 * REGS_HIGH <= THREADS * LAUNCH_REGS, "register split exceeds the launch");
-  static constexpr int SLOT_FLOATS = BM * D + 2 * BM;  // one partial: O rows, then m, then l
+  // One partial: O chunk-major ([D/4][BM] float4, so that the 32 rows of a
+  // warp read and write 512 contiguous bytes per chunk), then m, then l.
+  static constexpr int SLOT_FLOATS = BM * D + 2 * BM;
   static_assert(KST >= 2 && VST >= 2, "need at least two K and two V stages");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(O_COL0 + 2 * D <= TMEM_COLS, "TMEM budget");
@@ -632,11 +634,9 @@ __global__ void __launch_bounds__(384, 1)
           for (int c = 0; c < D / 16; ++c) {
             uint32_t oa[16], ob[16];
             tmem_load16(tOA + c * 16, oa);
-            tmem_load_wait16(oa);
-            if (hasB) {
-              tmem_load16(tOB + c * 16, ob);
-              tmem_load_wait16(ob);
-            }
+            if (hasB) tmem_load16(tOB + c * 16, ob);
+            tmem_load_wait16(oa);  // waits for both loads
+            if (hasB) tmem_load_wait16(ob);
             float* x = reinterpret_cast<float*>(oa);  // merged in place
 #pragma unroll
             for (int e = 0; e < 16; ++e)
@@ -653,10 +653,10 @@ __global__ void __launch_bounds__(384, 1)
                 }
               }
             } else {
-              float4* dst = reinterpret_cast<float4*>(slot + static_cast<size_t>(row) * D + c * 16);
+              float4* dst = reinterpret_cast<float4*>(slot) + static_cast<size_t>(4 * c) * BM + row;
 #pragma unroll
               for (int q4 = 0; q4 < 4; ++q4)
-                dst[q4] = make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]);
+                __stcg(dst + q4 * BM, make_float4(x[4 * q4], x[4 * q4 + 1], x[4 * q4 + 2], x[4 * q4 + 3]));
             }
           }
         }
@@ -678,34 +678,65 @@ __global__ void __launch_bounds__(384, 1)
           }
           asm volatile("bar.sync 3, 128;" ::: "memory");
           if (*s_last && ok) {
-            // the last piece of this unit to finish: merge every piece of it
+            // the last piece of this unit to finish: merge every piece of it.
+            // The loads of several slots are issued before any is used, so
+            // the merge costs a few L2 round trips, not one per chunk.
             __threadfence();
-            float mx = -INFINITY;
-            for (int gg = g_first; gg <= g_last; ++gg)
-              mx = fmaxf(mx, __ldcg(p.partials + static_cast<size_t>(gg + pc.u) * TR::SLOT_FLOATS + BM * D + row));
-            float Lt = 0.f;
-            for (int gg = g_first; gg <= g_last; ++gg) {
-              const float* sl = p.partials + static_cast<size_t>(gg + pc.u) * TR::SLOT_FLOATS;
-              Lt += __ldcg(sl + BM * D + BM + row) * ex2(__ldcg(sl + BM * D + row) - mx);
+            const int ns = g_last - g_first + 1;
+            const float* base = p.partials + static_cast<size_t>(g_first + pc.u) * TR::SLOT_FLOATS;
+            float mx = -INFINITY, Lt = 0.f;
+            for (int s0 = 0; s0 < ns; s0 += 4) {
+              float mv[4], lv[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const float* sl = base + static_cast<size_t>(s0 + k < ns ? s0 + k : s0) * TR::SLOT_FLOATS;
+                mv[k] = s0 + k < ns ? __ldcg(sl + BM * D + row) : -INFINITY;
+                lv[k] = s0 + k < ns ? __ldcg(sl + BM * D + BM + row) : 0.f;
+              }
+              // every piece holds at least one valid key, so its m is finite
+              const float nm = fmaxf(mx, fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])));
+              Lt *= ex2(mx - nm);
+#pragma unroll
+              for (int k = 0; k < 4; ++k) Lt += lv[k] * ex2(mv[k] - nm);
+              mx = nm;
             }
             const float inv = 1.0f / Lt;
 #pragma unroll 1
-            for (int c = 0; c < D / 8; ++c) {
-              float y[8];
+            for (int cb = 0; cb < D / 32; ++cb) {
+              float4 y[8];
 #pragma unroll
-              for (int e = 0; e < 8; ++e) y[e] = 0.f;
-              for (int gg = g_first; gg <= g_last; ++gg) {
-                const float* sl = p.partials + static_cast<size_t>(gg + pc.u) * TR::SLOT_FLOATS;
-                const float a = ex2(__ldcg(sl + BM * D + row) - mx) * inv;
-                const float4 v0 = __ldcg(reinterpret_cast<const float4*>(sl + static_cast<size_t>(row) * D + c * 8));
-                const float4 v1 =
-                    __ldcg(reinterpret_cast<const float4*>(sl + static_cast<size_t>(row) * D + c * 8 + 4));
-                y[0] += v0.x * a; y[1] += v0.y * a; y[2] += v0.z * a; y[3] += v0.w * a;
-                y[4] += v1.x * a; y[5] += v1.y * a; y[6] += v1.z * a; y[7] += v1.w * a;
+              for (int e = 0; e < 8; ++e) y[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+              for (int s0 = 0; s0 < ns; s0 += 2) {
+                float4 v[2][8];
+                float a[2];
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                  const bool valid = s0 + k < ns;
+                  const float* sl = base + static_cast<size_t>(valid ? s0 + k : s0) * TR::SLOT_FLOATS;
+                  a[k] = valid ? ex2(__ldcg(sl + BM * D + row) - mx) * inv : 0.f;
+                  const float4* src = reinterpret_cast<const float4*>(sl) + static_cast<size_t>(cb * 8) * BM + row;
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) v[k][e] = __ldcg(src + e * BM);
+                }
+#pragma unroll
+                for (int k = 0; k < 2; ++k)
+#pragma unroll
+                  for (int e = 0; e < 8; ++e) {
+                    y[e].x += v[k][e].x * a[k];
+                    y[e].y += v[k][e].y * a[k];
+                    y[e].z += v[k][e].z * a[k];
+                    y[e].w += v[k][e].w * a[k];
+                  }
               }
-              if (t < p.Tq)
-                store_chunk8<T>(static_cast<T*>(p.out) + ((static_cast<size_t>(b) * p.Tq + t) * p.H + h) * D + c * 8,
-                                y);
+              if (t < p.Tq) {
+                T* dst = static_cast<T*>(p.out) + ((static_cast<size_t>(b) * p.Tq + t) * p.H + h) * D + cb * 32;
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                  const float z[8] = {y[2 * q8].x, y[2 * q8].y, y[2 * q8].z, y[2 * q8].w,
+                                      y[2 * q8 + 1].x, y[2 * q8 + 1].y, y[2 * q8 + 1].z, y[2 * q8 + 1].w};
+                  store_chunk8<T>(dst + q8 * 8, z);
+                }
+              }
             }
             if (p.lse != nullptr && t < p.Tq)
               p.lse[(static_cast<size_t>(b) * p.H + h) * p.Tq + t] = (mx + log2f(Lt)) * 0.6931471805599453f;
