@@ -125,13 +125,16 @@ def test_append_fp8_codes_and_scales():
 
 # ---------------------------------------------------------------------------- attention
 def run_stream(w: W.Workload, frames, layer=0, rows_per_step=48, q_scale=1.0, check_lse=True, dtype=None,
-               B=None, mean_abs=1e-3, lse_rel=1e-3, max_rel=1e-2, scale=None):
+               B=None, mean_abs=1e-3, lse_rel=1e-3, max_rel=1e-2, scale=None, k_scale=None, no_rope=False):
     """Append + attend frame by frame (or chunk by chunk); compare sampled rows
     (all rows when the step is small) with the oracle stream."""
     B = B or w.B
     cache = swa.KVCache(B, w.H, w.D, w.N, dtype or w.dtype)
-    rope = rope_of(w)
-    oracles = [StreamOracle(w.H, w.D, w.grid_h, w.grid_w, omega_of(w), w.pairs, w.t_offset) for _ in range(B)]
+    # no_rope: Q and K are passed as already rotated (rope descriptor NULL);
+    # the oracle then rotates by angle 0 (all frequencies zero)
+    rope = None if no_rope else rope_of(w)
+    om = np.zeros_like(omega_of(w)) if no_rope else omega_of(w)
+    oracles = [StreamOracle(w.H, w.D, w.grid_h, w.grid_w, om, w.pairs, w.t_offset) for _ in range(B)]
     c = w.query_frames
     worst = (0.0, 0.0)
     for f0 in frames:
@@ -141,6 +144,8 @@ def run_stream(w: W.Workload, frames, layer=0, rows_per_step=48, q_scale=1.0, ch
         v = torch.cat([p[2] for p in parts], 0)
         if q_scale != 1.0:
             q = (q.float() * q_scale).to(q.dtype)
+        if k_scale is not None:
+            k = (k.float() * k_scale(f0)).to(k.dtype)
         swa.kvcache_append(cache, k.cuda(), v.cuda(), f0, rope)
         lse = torch.empty(B, w.H, q.shape[1], device="cuda", dtype=torch.float32)
         out = swa.sink_window_attention(q.cuda(), cache, f0, rope, lse=lse, softmax_scale=scale or 0.0)
@@ -192,6 +197,19 @@ def test_attention_wan_warmup_and_steady():
 def test_attention_wan_peaked():
     w = W.WAN
     run_stream(w, [0, 1, 2, 3], rows_per_step=24, q_scale=8.0)
+
+
+def test_attention_wan_growing_logits():
+    """Keys of later frames scaled up (K x (1 + f), Q x 4): a row's logit max
+    grows by far more than 2^8 (in the exp2 domain) between the first key
+    tiles of a piece and the later ones, so the kernel's rescale (O and the
+    row sum scaled to the new max, P computed again from S) runs on most rows.
+    Q and K go in already rotated (no RoPE in the kernels), so the inputs the
+    kernel multiplies are exactly the oracle's: with logits up to ~20, a
+    rotation rounded to bf16 would move them by ~2^-9 * |logit|, more than
+    the bar allows for a softmax this sharp."""
+    w = W.WAN
+    run_stream(w, range(5), rows_per_step=24, q_scale=4.0, k_scale=lambda f: 1.0 + f, no_rope=True)
 
 
 def test_attention_chunk_jitter():
