@@ -310,7 +310,8 @@ def run_ours(args, rank, world, local_rank):
     avg_attn_s = (sum(attn_ms) / len(attn_ms)) / 1e3
     fl = attention_flops(w)
     achieved = fl / avg_attn_s / 1e12
-    traffic = load_traffic()
+    # the timed launch is the fused append + attention in the default stream
+    traffic = load_traffic("attention_fused_stream.md" if fused else "attention_wan_single_layer.md")
     recache_ms = [a.elapsed_time(b) for a, b in rev[2]]
     rc_layer_s = (sum(recache_ms) / len(recache_ms)) / 1e3 / w.layers
     rc_flops = 2.0 * (w.slots * w.N) * w.dm * (2 * w.H * w.D)
@@ -430,11 +431,11 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def load_traffic():
-    """DRAM bytes (read + write) per attention launch from the committed ncu
+def load_traffic(profile: str = "attention_wan_single_layer.md"):
+    """DRAM bytes (read + write) per attention launch from a committed ncu
     summary — only while the kernel sources still hash to the captured
     version; otherwise null."""
-    p = os.path.join(ROOT, "profiles", "attention_wan_single_layer.md")
+    p = os.path.join(ROOT, "profiles", profile)
     if not os.path.exists(p):
         return None
     text = open(p).read()
