@@ -31,7 +31,7 @@ def rmsnorm(x: np.ndarray, gamma: np.ndarray, eps: float) -> np.ndarray:
 
 def recache_frame(x: np.ndarray, wk: np.ndarray, wv: np.ndarray, gamma: np.ndarray,
                   eps: float, frame: int, H: int, D: int, grid_h: int, grid_w: int,
-                  omega: np.ndarray, pairs, t_offset: int = 0):
+                  omega: np.ndarray, pairs, t_offset: int = 0, t_scale: float = 1.0):
     """Recomputed (rotated K, V) of one frame from its hidden states x [N, Dm].
 
     Returns k_rot [N, H, D] and v [N, H, D]."""
@@ -39,5 +39,5 @@ def recache_frame(x: np.ndarray, wk: np.ndarray, wv: np.ndarray, gamma: np.ndarr
     kp = x @ np.asarray(wk, dtype=np.float64)
     vp = x @ np.asarray(wv, dtype=np.float64)
     k = rmsnorm(kp, gamma, eps).reshape(-1, H, D)
-    t, r, c = token_positions(frame, grid_h, grid_w, t_offset)
+    t, r, c = token_positions(frame, grid_h, grid_w, t_offset, t_scale)
     return rope_3d(k, t, r, c, omega, pairs), vp.reshape(-1, H, D)

@@ -12,6 +12,15 @@ Sources
   The jitter is applied to the temporal band only (d_time), a reading stated
   for the chunk workload; the spatial bands keep theta0.
 
+* LoL review, "Core innovation": the phase concentration of the RoPE
+  components at a relative offset Delta is measured by the phase-coherence
+  kernel C(Delta) = (1/K) sum_i exp(j omega_i Delta); it peaks where the sink
+  frames collapse. Reading: for the temporal offset between frames the K
+  components are the K = pairs_t frequencies of a head's temporal band.
+* LoL review, "Motivation" and results table: position interpolation (PI) is
+  the baseline that compresses positions; reading: the temporal position
+  (t_offset + f) is multiplied by a factor t_scale (1 = plain RoPE).
+
 Layout reading: rotary pairs are adjacent channels (2j, 2j+1) of each head;
 the head dimension is split into a temporal band of ``pt`` pairs followed by
 ``ph`` pairs for the grid row and ``pw`` pairs for the grid column. Inside a
@@ -69,13 +78,27 @@ def rotate_pairs(x: np.ndarray, angle: np.ndarray) -> np.ndarray:
     return out
 
 
-def token_positions(frame: int, grid_h: int, grid_w: int, t_offset: int = 0):
+def token_positions(frame: int, grid_h: int, grid_w: int, t_offset: int = 0, t_scale: float = 1.0):
     """(t, h, w) of every token of one latent frame, tokens in row-major (h, w)
-    order; t = t_offset + absolute frame index."""
+    order; t = (t_offset + absolute frame index) * t_scale (t_scale != 1: position
+    interpolation of the temporal axis)."""
     r = np.repeat(np.arange(grid_h), grid_w)
     c = np.tile(np.arange(grid_w), grid_h)
-    t = np.full(grid_h * grid_w, t_offset + frame)
+    t = np.full(grid_h * grid_w, float(t_offset + frame) * float(t_scale))
     return t.astype(np.float64), r.astype(np.float64), c.astype(np.float64)
+
+
+def phase_coherence(omega: np.ndarray, deltas) -> np.ndarray:
+    """C(Delta) = (1/K) * sum_{i<K} exp(j * omega_i * Delta) for every Delta
+    (LoL review, "Core innovation"), omega [K] (one head's components).
+    Returns complex128 [len(deltas)]."""
+    omega = np.asarray(omega, dtype=np.float64)
+    deltas = np.asarray(deltas, dtype=np.float64)
+    K = omega.shape[0]
+    out = np.zeros(deltas.shape[0], dtype=np.complex128)
+    for i in range(K):  # one component at a time, as the sum is written
+        out += np.exp(1j * omega[i] * deltas)
+    return out / K
 
 
 def rope_3d(x: np.ndarray, pos_t, pos_h, pos_w, omega: np.ndarray, pairs) -> np.ndarray:
@@ -93,7 +116,7 @@ def rope_3d(x: np.ndarray, pos_t, pos_h, pos_w, omega: np.ndarray, pairs) -> np.
 
 
 def rope_frames(x: np.ndarray, first_frame: int, grid_h: int, grid_w: int, omega, pairs,
-                t_offset: int = 0) -> np.ndarray:
+                t_offset: int = 0, t_scale: float = 1.0) -> np.ndarray:
     """RoPE of x [B, F*N, H, D] holding consecutive frames first_frame.. first_frame+F-1."""
     x = np.asarray(x, dtype=np.float64)
     B, T, H, D = x.shape
@@ -101,7 +124,7 @@ def rope_frames(x: np.ndarray, first_frame: int, grid_h: int, grid_w: int, omega
     F = T // N
     out = np.empty_like(x)
     for fi in range(F):
-        t, r, c = token_positions(first_frame + fi, grid_h, grid_w, t_offset)
+        t, r, c = token_positions(first_frame + fi, grid_h, grid_w, t_offset, t_scale)
         for b in range(B):
             out[b, fi * N:(fi + 1) * N] = rope_3d(x[b, fi * N:(fi + 1) * N], t, r, c, omega, pairs)
     return out

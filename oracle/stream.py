@@ -28,20 +28,21 @@ from .window import attended_frames
 
 class StreamOracle:
     def __init__(self, H: int, D: int, grid_h: int, grid_w: int, omega: np.ndarray, pairs,
-                 t_offset: int = 0, n_sink: int = 3, n_local: int = 9):
+                 t_offset: int = 0, n_sink: int = 3, n_local: int = 9, t_scale: float = 1.0):
         self.H, self.D = H, D
         self.grid_h, self.grid_w = grid_h, grid_w
         self.N = grid_h * grid_w
         self.omega = np.asarray(omega, dtype=np.float64)
         self.pairs = tuple(pairs)
         self.t_offset = t_offset
+        self.t_scale = t_scale
         self.n_sink, self.n_local = n_sink, n_local
         self.k: Dict[int, np.ndarray] = {}   # frame -> rotated K [N, H, D]
         self.v: Dict[int, np.ndarray] = {}   # frame -> V [N, H, D]
         self.last = -1
 
     def _rot(self, x: np.ndarray, frame: int) -> np.ndarray:
-        t, r, c = token_positions(frame, self.grid_h, self.grid_w, self.t_offset)
+        t, r, c = token_positions(frame, self.grid_h, self.grid_w, self.t_offset, self.t_scale)
         return rope_3d(x, t, r, c, self.omega, self.pairs)
 
     def append(self, first_frame: int, k: np.ndarray, v: np.ndarray, replace: bool = False) -> None:
@@ -100,6 +101,6 @@ class StreamOracle:
         frames = [g for g in attended_frames(switch_frame - 1, self.n_sink, self.n_local)]
         for g in frames:
             k, v = recache_frame(x_by_frame[g], wk, wv, gamma, eps, g, self.H, self.D,
-                                 self.grid_h, self.grid_w, self.omega, self.pairs, self.t_offset)
+                                 self.grid_h, self.grid_w, self.omega, self.pairs, self.t_offset, self.t_scale)
             self.k[g] = k
             self.v[g] = v

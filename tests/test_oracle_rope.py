@@ -141,3 +141,74 @@ def test_token_positions_row_major():
     assert np.all(t == 2007)
     assert list(r[:7]) == [0, 0, 0, 0, 0, 0, 1] and list(c[:7]) == [0, 1, 2, 3, 4, 5, 0]
     assert r[-1] == 3 and c[-1] == 5
+
+
+# ---------------------------------------------------------------- phase coherence and position interpolation
+def test_phase_coherence_special_values():
+    """C(0) = 1, |C| <= 1, C(-D) = conj C(D); one component is a pure phase."""
+    om = rope.band_frequencies(10000.0, 22)
+    d = np.arange(-300, 301, dtype=np.float64)
+    c = rope.phase_coherence(om, d)
+    assert c[300] == pytest.approx(1.0, abs=1e-15)
+    assert np.all(np.abs(c) <= 1.0 + 1e-12)
+    assert np.allclose(c[::-1], np.conj(c), atol=1e-13)
+    one = rope.phase_coherence(om[:1], d)
+    assert np.allclose(one, np.cos(d) + 1j * np.sin(d), atol=1e-13)
+
+
+def test_phase_coherence_harmonic_closed_form():
+    """Components i*w0 (i = 0..K-1): the sum is a geometric series,
+    C(D) = (1 - z^K) / (K (1 - z)) with z = e^{j w0 D}, and C = 1 whenever
+    w0 D is a multiple of 2 pi (every component back in phase)."""
+    K, w0 = 7, 0.37
+    om = w0 * np.arange(K, dtype=np.float64)
+    d = np.array([0.5, 1.0, 2.5, 10.0, 123.4])
+    z = np.exp(1j * w0 * d)
+    want = (1 - z ** K) / (K * (1 - z))
+    assert np.allclose(rope.phase_coherence(om, d), want, atol=1e-13)
+    period = 2 * math.pi / w0
+    assert np.allclose(rope.phase_coherence(om, [period, 3 * period]), 1.0, atol=1e-12)
+
+
+def test_phase_coherence_decorrelates_over_long_offsets():
+    """For RoPE's geometric frequencies the components drift apart: averaged
+    over many offsets, |C|^2 approaches 1/K (the components' phases behave as
+    independent), far below the 1 at D = 0."""
+    om = rope.band_frequencies(10000.0, 22)
+    d = np.arange(1000, 200000, 7, dtype=np.float64)
+    m2 = np.mean(np.abs(rope.phase_coherence(om, d)) ** 2)
+    assert 0.5 / 22 < m2 < 2.0 / 22
+
+
+def test_phase_coherence_jitter_breaks_alignment():
+    """Heads with different jittered bases (LoL "Method steps") have different
+    C(D) away from D = 0; with sigma = 0 every head has the same curve."""
+    eps = W.jitter_eps(3, 4).astype(np.float64)
+    om = rope.head_frequencies(4, (22, 21, 21), 10000.0, 0.8, eps)
+    om0 = rope.head_frequencies(4, (22, 21, 21), 10000.0, 0.0, None)
+    d = np.arange(1, 500, dtype=np.float64)
+    cj = [rope.phase_coherence(om[h, :22], d) for h in range(4)]
+    c0 = [rope.phase_coherence(om0[h, :22], d) for h in range(4)]
+    assert all(np.array_equal(c0[0], c) for c in c0[1:])
+    assert all(np.max(np.abs(cj[0] - c)) > 0.1 for c in cj[1:])
+
+
+def test_position_interpolation_pins():
+    """t_scale = 1 is plain RoPE; with t_scale = 1/2 frame 2f sits at the
+    position of frame f; the relative identity holds at scaled positions."""
+    rng = np.random.default_rng(5)
+    pairs = (12, 10, 10)
+    om = rope.head_frequencies(2, pairs, 10000.0)
+    x = rng.standard_normal((1, 24, 2, 64))
+    a = rope.rope_frames(x, 7, 4, 6, om, pairs)
+    b = rope.rope_frames(x, 7, 4, 6, om, pairs, t_scale=1.0)
+    assert np.array_equal(a, b)
+    c = rope.rope_frames(x, 14, 4, 6, om, pairs, t_scale=0.5)
+    assert np.allclose(c, a, atol=1e-14)
+    # <R(s m) q, R(s n) k> = <q, R(s (n - m)) k> per pair
+    q, k = rng.standard_normal(64), rng.standard_normal(64)
+    s, m, n = 0.3, 11.0, 29.0
+    w = om[0, 0]
+    lhs = rope.rotate_pairs(q[:2], s * m * w) @ rope.rotate_pairs(k[:2], s * n * w)
+    rhs = q[:2] @ rope.rotate_pairs(k[:2], s * (n - m) * w)
+    assert lhs == pytest.approx(rhs, abs=1e-12)
