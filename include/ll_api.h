@@ -46,7 +46,7 @@
 extern "C" {
 #endif
 
-#define LL_ABI_VERSION 1
+#define LL_ABI_VERSION 2
 #define LL_MAX_HEADS 64
 
 typedef enum ll_status {
@@ -73,7 +73,12 @@ typedef enum ll_dtype {
  * pairs_h pairs for the grid row and pairs_w for the grid column; inside a
  * band of P pairs, i = 0..P-1 and d = 2P. The temporal band of head h uses
  * base theta0 * (1 + sigma_t * eps_h[h]); the two spatial bands use theta0.
- * Token (frame f, row r, column c) sits at position (t_offset + f, r, c).
+ * Token (frame f, row r, column c) sits at position ((t_offset + f) * s, r, c)
+ * with s = t_scale: position interpolation, the baseline that the LoL review
+ * compares against ("Motivation" and results table: PI compresses positions),
+ * for s in (0, 1); s = 0 or 1 gives plain RoPE, so a zero-initialised field
+ * keeps the ABI-1 behaviour. Validation: LL_ERR_INVALID_ARG for s outside
+ * [0, 1].
  */
 typedef struct ll_rope_desc {
   int pairs_t, pairs_h, pairs_w;  /* pairs per axis; pairs_t + pairs_h + pairs_w = D/2 */
@@ -82,6 +87,7 @@ typedef struct ll_rope_desc {
   const float* eps_h;             /* HOST pointer to H draws in [-1, 1], or NULL for no jitter */
   int grid_h, grid_w;             /* token grid of one latent frame */
   long long t_offset;             /* temporal position of frame 0 */
+  double t_scale;                 /* temporal position factor in [0, 1]; 0 or 1 = no interpolation */
 } ll_rope_desc;
 
 /*
@@ -210,6 +216,25 @@ ll_status ll_append_and_attend(const ll_kvcache* cache, const void* k, const voi
                                ll_dtype dtype, long long first_frame, int n_frames,
                                const ll_rope_desc* rope, float softmax_scale, void* out, float* lse,
                                void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Phase-coherence kernel of the temporal RoPE band (LoL review, "Core
+ * innovation": the phase concentration C(D) = (1/K) sum_{i=1..K}
+ * exp(j w_i D) peaks at the offsets where the sink frames collapse, and the
+ * per-head jitter of "Method steps" spreads those peaks across heads).
+ * For every head h and frame offset D = delta0 .. delta0 + n_delta - 1:
+ *   out[h][k] = (re, im) of (1/K) sum_{i<K} exp(j * w_{h,i} * s * D)
+ * with K = rope->pairs_t, w_{h,i} = base_h^(-i/K) the temporal-band
+ * frequencies of head h (base_h = theta0 (1 + sigma_t eps_h[h])) and
+ * s = t_scale (1 when 0). The spatial bands do not enter (reading: D is an
+ * offset between frames). Evaluated in fp64, stored as fp32.
+ * out: DEVICE [H][n_delta][2] floats, caller-owned, 8-byte aligned.
+ * Errors: LL_ERR_INVALID_ARG for a NULL pointer, H outside [1, LL_MAX_HEADS],
+ * n_delta < 1, pairs_t < 1, offsets beyond +-2^40 or an invalid rope
+ * descriptor; LL_ERR_UNSUPPORTED when H * n_delta >= 2^31.
+ */
+ll_status ll_phase_coherence(const ll_rope_desc* rope, int H, long long delta0, int n_delta, float* out,
+                             void* stream);
 
 /*
  * Allocation-free variant of ll_sink_window_attention (the pages have no

@@ -21,12 +21,13 @@ LIB_PATH = os.path.join(_HERE, "libll_swa.so")
 LL_OK, LL_ERR_INVALID_ARG, LL_ERR_UNSUPPORTED, LL_ERR_CUDA, LL_ERR_TIMEOUT = range(5)
 LL_F32, LL_BF16, LL_FP8_E4M3 = 0, 1, 2
 MAX_HEADS = 64
+ABI_VERSION = 2
 
 EXPORTED = (
     "ll_abi_version", "ll_last_error", "ll_slot_of_frame", "ll_device_error", "ll_rope_apply",
     "ll_kvcache_append", "ll_sink_window_attention_workspace_bytes", "ll_sink_window_attention",
     "ll_kv_recache_workspace_bytes", "ll_kv_recache", "ll_sink_window_attention_noalloc",
-    "ll_append_and_attend_workspace_bytes", "ll_append_and_attend",
+    "ll_append_and_attend_workspace_bytes", "ll_append_and_attend", "ll_phase_coherence",
 )
 NOALLOC_SCRATCH_BYTES = 48 * 1024 * 1024
 
@@ -41,7 +42,7 @@ class RopeDescC(ctypes.Structure):
     _fields_ = [("pairs_t", ctypes.c_int), ("pairs_h", ctypes.c_int), ("pairs_w", ctypes.c_int),
                 ("theta0", ctypes.c_double), ("sigma_t", ctypes.c_double),
                 ("eps_h", ctypes.POINTER(ctypes.c_float)), ("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int),
-                ("t_offset", ctypes.c_longlong)]
+                ("t_offset", ctypes.c_longlong), ("t_scale", ctypes.c_double)]
 
 
 class KVCacheC(ctypes.Structure):
@@ -79,6 +80,7 @@ def lib() -> ctypes.CDLL:
         L.ll_append_and_attend_workspace_bytes.argtypes = [cp, i]
         L.ll_append_and_attend_workspace_bytes.restype = sz
         L.ll_append_and_attend.argtypes = [cp, vp, vp, vp, i, ll_, i, rp, f, vp, vp, vp, sz, vp]
+        L.ll_phase_coherence.argtypes = [rp, i, ll_, i, vp, vp]
         for name in EXPORTED[2:]:
             if not name.endswith("_workspace_bytes"):
                 getattr(L, name).restype = i
@@ -127,6 +129,7 @@ class Rope:
     sigma_t: float = 0.0
     eps: Optional[Sequence[float]] = None
     t_offset: int = 0
+    t_scale: float = 1.0   # position interpolation of the temporal axis (1: plain RoPE)
 
     def to_c(self) -> RopeDescC:
         r = RopeDescC()
@@ -138,6 +141,7 @@ class Rope:
             r._eps_keepalive = arr  # noqa: keep the host array alive with the struct
             r.eps_h = ctypes.cast(arr, ctypes.POINTER(ctypes.c_float))
         r.grid_h, r.grid_w, r.t_offset = int(self.grid_h), int(self.grid_w), int(self.t_offset)
+        r.t_scale = float(self.t_scale)
         return r
 
 
@@ -315,3 +319,15 @@ def kv_recache(cache: KVCache, x: torch.Tensor, wk: torch.Tensor, wv: torch.Tens
     _check(lib().ll_kv_recache(ctypes.byref(cache.to_c()), _ptr(x), x.shape[-1], _ptr(wk), _ptr(wv), _ptr(gamma),
                                float(rms_eps), frames, n, _rope_ref(rope), _ptr(workspace), ws_bytes,
                                _stream(stream)))
+
+
+def phase_coherence(rope: Rope, H: int, delta0: int, n_delta: int, out: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """C_h(D) of the temporal RoPE band for D = delta0 .. delta0 + n_delta - 1
+    (ll_phase_coherence): float32 [H, n_delta, 2] (real, imaginary) on the
+    current CUDA device."""
+    if out is None:
+        out = torch.empty((H, n_delta, 2), dtype=torch.float32, device="cuda")
+    _check(lib().ll_phase_coherence(ctypes.byref(rope.to_c()), H, int(delta0), int(n_delta), _ptr(out),
+                                    _stream(stream)))
+    return out

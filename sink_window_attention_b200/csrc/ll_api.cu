@@ -60,12 +60,15 @@ ll_status make_rope(const ll_rope_desc* r, int H, int D, long long t_first, ll::
   if (r->grid_h < 1 || r->grid_w < 1) return fail(LL_ERR_INVALID_ARG, "rope grid must be at least 1x1");
   if (H > ll::kMaxHeads) return fail(LL_ERR_INVALID_ARG, "H = %d exceeds %d", H, ll::kMaxHeads);
   if (r->t_offset < 0) return fail(LL_ERR_INVALID_ARG, "rope t_offset must be >= 0");
+  if (!(r->t_scale >= 0.0 && r->t_scale <= 1.0))
+    return fail(LL_ERR_INVALID_ARG, "rope t_scale must lie in [0, 1] (0 and 1: no interpolation)");
   out->enabled = 1;
   out->pt = r->pairs_t;
   out->ph = r->pairs_h;
   out->pw = r->pairs_w;
   out->grid_w = r->grid_w;
   out->t_first = r->t_offset + t_first;
+  out->t_scale = r->t_scale > 0.0 ? static_cast<float>(r->t_scale) : 1.0f;
   out->theta0 = r->theta0;
   out->sigma = r->eps_h ? r->sigma_t : 0.0;
   for (int h = 0; h < H; ++h) {
@@ -522,6 +525,34 @@ ll_status ll_append_and_attend(const ll_kvcache* cache, const void* k, const voi
   if (!f32)
     return launch_attention<ll::AttnTraits<64, __nv_bfloat16>>(p, cache, S, workspace, workspace_bytes, s, true);
   return launch_attention<ll::AttnTraits<64, float>>(p, cache, S, workspace, workspace_bytes, s, true);
+}
+
+ll_status ll_phase_coherence(const ll_rope_desc* rope, int H, long long delta0, int n_delta, float* out,
+                             void* stream) {
+  g_last_error.clear();
+  if (rope == nullptr || out == nullptr) return fail(LL_ERR_INVALID_ARG, "rope and out must be non-NULL");
+  if ((reinterpret_cast<uintptr_t>(out) & 7u) != 0) return fail(LL_ERR_INVALID_ARG, "out must be 8-byte aligned");
+  if (H < 1 || H > ll::kMaxHeads) return fail(LL_ERR_INVALID_ARG, "H = %d must lie in [1, %d]", H, ll::kMaxHeads);
+  if (n_delta < 1) return fail(LL_ERR_INVALID_ARG, "n_delta must be >= 1");
+  if (rope->pairs_t < 1) return fail(LL_ERR_INVALID_ARG, "the temporal band needs pairs_t >= 1");
+  const long long lim = 1LL << 40;  // offsets far beyond any stream; keeps delta * t_scale exact in fp64
+  if (delta0 < -lim || delta0 > lim - n_delta)
+    return fail(LL_ERR_INVALID_ARG, "offsets must lie within +-2^40 frames");
+  if (static_cast<long long>(H) * n_delta >= (1LL << 31))
+    return fail(LL_ERR_UNSUPPORTED, "H * n_delta too large for one call");
+  ll::PhaseParams p{};
+  const int D = 2 * (rope->pairs_t + rope->pairs_h + rope->pairs_w);
+  ll_status st = make_rope(rope, H, D, 0, &p.rp);
+  if (st != LL_OK) return st;
+  p.t_scale = rope->t_scale > 0.0 ? rope->t_scale : 1.0;
+  p.delta0 = delta0;
+  p.H = H;
+  p.n = n_delta;
+  p.out = reinterpret_cast<float2*>(out);
+  const long long threads = static_cast<long long>(H) * n_delta;
+  ll::phase_coherence_kernel<<<static_cast<unsigned>((threads + 255) / 256), 256, 0,
+                               static_cast<cudaStream_t>(stream)>>>(p);
+  return check_launch("phase_coherence_kernel");
 }
 
 }  // extern "C"

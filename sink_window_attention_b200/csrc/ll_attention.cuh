@@ -151,7 +151,7 @@ __device__ __forceinline__ void rope_q_tile_inplace(uint8_t* sQ, const AttnParam
         x[2 * i] = f.x;
         x[2 * i + 1] = f.y;
       }
-      rotate_chunk8(x, e8 * 4, static_cast<float>(p.rp.t_first + fi), static_cast<float>(rr),
+      rotate_chunk8(x, e8 * 4, temporal_pos(p.rp, fi), static_cast<float>(rr),
                     static_cast<float>(cc), om, p.rp.pt, pth);
       *ptr = make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]), pack_bf16(x[6], x[7]));
     } else {
@@ -160,7 +160,7 @@ __device__ __forceinline__ void rope_q_tile_inplace(uint8_t* sQ, const AttnParam
       const float4 a = *p0, b = *p1;
       x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
       x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-      rotate_chunk8(x, e8 * 4, static_cast<float>(p.rp.t_first + fi), static_cast<float>(rr),
+      rotate_chunk8(x, e8 * 4, temporal_pos(p.rp, fi), static_cast<float>(rr),
                     static_cast<float>(cc), om, p.rp.pt, pth);
       *p0 = make_float4(x[0], x[1], x[2], x[3]);
       *p1 = make_float4(x[4], x[5], x[6], x[7]);

@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(256, 2)
     const int slot = live ? t / p.N : 0;
     const int n = live ? t - slot * p.N : 0;
     const int gw = p.rp.grid_w > 0 ? p.rp.grid_w : 1;
-    const float pos_t = static_cast<float>(p.rp.t_first + (live ? p.slot_frame[slot] : 0));
+    const float pos_t = temporal_pos(p.rp, live ? p.slot_frame[slot] : 0);
     const float pos_r = static_cast<float>(n / gw);
     const float pos_c = static_cast<float>(n % gw);
     const size_t crow = static_cast<size_t>(b) * p.S * p.N + t;  // cache token row

@@ -15,12 +15,13 @@ namespace ll {
 constexpr int kMaxHeads = 64;
 
 // RoPE parameters as the kernels receive them. Position of token n of the
-// i-th frame in a tensor: (t_first + i, n / grid_w, n % grid_w).
+// i-th frame in a tensor: ((t_first + i) * t_scale, n / grid_w, n % grid_w).
 struct RopeParams {
   int enabled;
   int pt, ph, pw;          // pairs per band (t, h, w); pt + ph + pw = D/2
   int grid_w;
-  long long t_first;       // temporal position of the tensor's first frame (t_offset included)
+  float t_scale;           // temporal position factor (position interpolation; 1 = plain RoPE)
+  long long t_first;       // index of the tensor's first frame, t_offset included
   double theta0;
   double sigma;
   float eps[kMaxHeads];    // per-head jitter draws (0 when there is no jitter)
@@ -46,6 +47,12 @@ __device__ __forceinline__ float omega_of(const RopeParams& rp, int h, int j) {
     pairs = rp.pw;
   }
   return exp2f(-(static_cast<float>(i) / static_cast<float>(pairs)) * log2f(base));
+}
+
+// Temporal position of the i-th frame of a tensor: (t_first + i) * t_scale
+// (the frame index is exact in fp32 below 2^24; t_scale = 1 leaves it exact).
+__device__ __forceinline__ float temporal_pos(const RopeParams& rp, long long i) {
+  return static_cast<float>(rp.t_first + i) * rp.t_scale;
 }
 
 // omega[hh * P + j] for heads h0 .. h0+nh-1, built by the whole block.
@@ -144,6 +151,40 @@ __device__ __forceinline__ uint2 encode_chunk8_e4m3(const float (&x)[8], float s
 }
 
 // ---------------------------------------------------------------------------
+// Phase-coherence kernel of a head's temporal band (LoL review, "Core
+// innovation"): C_h(D) = (1/K) sum_{i<K} exp(j omega_{h,i} s D) with
+// K = pt, omega_{h,i} = base_h^(-i/pt), base_h = theta0 (1 + sigma eps_h),
+// s = t_scale, for the frame offsets D = delta0 .. delta0 + n - 1. One thread
+// per (head, offset); frequencies, angles and the sum in fp64 (angles reach
+// 1e5 rad and more), stored as fp32 (re, im).
+// ---------------------------------------------------------------------------
+struct PhaseParams {
+  RopeParams rp;
+  double t_scale;
+  long long delta0;
+  int H, n;
+  float2* out;  // [H][n]
+};
+
+__global__ void __launch_bounds__(256) phase_coherence_kernel(const PhaseParams p) {
+  const long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<long long>(p.H) * p.n) return;
+  const int h = static_cast<int>(idx / p.n);
+  const int k = static_cast<int>(idx - static_cast<long long>(h) * p.n);
+  const double lb = log2(p.rp.theta0 * (1.0 + p.rp.sigma * static_cast<double>(p.rp.eps[h])));
+  const double d = static_cast<double>(p.delta0 + k) * p.t_scale;
+  double re = 0.0, im = 0.0;
+  for (int i = 0; i < p.rp.pt; ++i) {
+    const double w = exp2(-(static_cast<double>(i) / p.rp.pt) * lb);
+    double sn, cs;
+    sincos(w * d, &sn, &cs);
+    re += cs;
+    im += sn;
+  }
+  p.out[idx] = make_float2(static_cast<float>(re / p.rp.pt), static_cast<float>(im / p.rp.pt));
+}
+
+// ---------------------------------------------------------------------------
 // K0: in-place RoPE of x [B][F*N][H][D].
 // ---------------------------------------------------------------------------
 struct RopeApplyParams {
@@ -175,7 +216,7 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(const RopeApplyParams p
     float v[8];
     T* ptr = x + static_cast<size_t>(row) * p.D + c * 8;
     load_chunk8<T>(ptr, v);
-    rotate_chunk8(v, c * 4, static_cast<float>(p.rp.t_first + fi), static_cast<float>(r),
+    rotate_chunk8(v, c * 4, temporal_pos(p.rp, fi), static_cast<float>(r),
                   static_cast<float>(col), s_omega + h * P, p.rp.pt, pth);
     store_chunk8<T>(ptr, v);
   }
@@ -233,7 +274,7 @@ __device__ __forceinline__ void build_append_tables(float* s_omega, float* s_tcs
     const int f = idx / (p.H * p.rp.pt), rem = idx - f * (p.H * p.rp.pt);
     const int h = rem / p.rp.pt, j = rem - h * p.rp.pt;
     float sn, cs;
-    sincos_reduced(static_cast<float>(p.rp.t_first + f) * s_omega[h * P + j], sn, cs);
+    sincos_reduced(temporal_pos(p.rp, f) * s_omega[h * P + j], sn, cs);
     s_tcs[2 * idx] = cs;
     s_tcs[2 * idx + 1] = sn;
   }

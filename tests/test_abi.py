@@ -31,7 +31,7 @@ def test_exports_every_declared_symbol(L):
     for n in names:
         assert hasattr(L, n), n
     assert set(names) == set(swa.EXPORTED)
-    assert swa.abi_version() == 1
+    assert swa.abi_version() == swa.ABI_VERSION == 2
 
 
 @pytest.mark.parametrize("n_sink,n_local", [(3, 9), (0, 5), (2, 1), (4, 12)])
@@ -160,3 +160,25 @@ def test_fused_append_attention_validation(L):
         st = _fused(L, **kw)
         assert st == swa.LL_ERR_INVALID_ARG, (kw, st)
         assert swa.last_error() != ""
+
+
+def test_phase_coherence_and_position_interpolation_validation(L):
+    """ll_phase_coherence and the rope descriptor's t_scale are checked on the
+    host; every rejected call returns before a launch."""
+    out = 1 << 22
+    assert L.ll_phase_coherence(None, 12, 0, 16, out, None) == swa.LL_ERR_INVALID_ARG
+    r = _rope()
+    assert L.ll_phase_coherence(ctypes.byref(r), 12, 0, 16, None, None) == swa.LL_ERR_INVALID_ARG
+    assert L.ll_phase_coherence(ctypes.byref(r), 12, 0, 16, out + 4, None) == swa.LL_ERR_INVALID_ARG  # alignment
+    assert L.ll_phase_coherence(ctypes.byref(r), 0, 0, 16, out, None) == swa.LL_ERR_INVALID_ARG
+    assert L.ll_phase_coherence(ctypes.byref(r), 65, 0, 16, out, None) == swa.LL_ERR_INVALID_ARG
+    assert L.ll_phase_coherence(ctypes.byref(r), 12, 0, 0, out, None) == swa.LL_ERR_INVALID_ARG
+    assert L.ll_phase_coherence(ctypes.byref(r), 12, 1 << 41, 16, out, None) == swa.LL_ERR_INVALID_ARG
+    assert L.ll_phase_coherence(ctypes.byref(_rope(pairs_t=0, pairs_h=32)), 12, 0, 16, out,
+                                None) == swa.LL_ERR_INVALID_ARG
+    assert L.ll_phase_coherence(ctypes.byref(r), 64, 0, 1 << 26, out, None) == swa.LL_ERR_UNSUPPORTED
+    for bad in (-0.5, 1.5, float("nan")):
+        rb = _rope(t_scale=bad)
+        assert L.ll_phase_coherence(ctypes.byref(rb), 12, 0, 16, out, None) == swa.LL_ERR_INVALID_ARG
+        assert "t_scale" in swa.last_error()
+        assert _attn(L, _cache(), rope=rb, ws=1 << 24, ws_bytes=1 << 30) == swa.LL_ERR_INVALID_ARG

@@ -68,6 +68,28 @@ def test_rope_apply(name):
     assert_parity(np64(xg), ref, max_rel=tol, mean_abs=1e-3 if w.dtype != "f32" else 1e-6, what="rope")
 
 
+@pytest.mark.parametrize("name", ["tiny", "chunk"])
+def test_rope_position_interpolation(name):
+    """Position interpolation (t_scale): against the oracle at scale 1/4, and
+    bit-identical to plain RoPE where the positions coincide (scale 1/2 at
+    frame 2f is plain RoPE at frame f; the offset is scaled too, so it is 0
+    here)."""
+    w = W.replace(W.WORKLOADS[name], t_offset=0)
+    x, _, _ = W.qkv_frames(w, 8, 3, 2)
+    r = rope_of(w)
+    r.t_scale = 0.25
+    xg = x.cuda()
+    swa.rope_apply(xg, 9, r)
+    ref = orope.rope_frames(np64(x), 9, w.grid_h, w.grid_w, omega_of(w), w.pairs, 0, t_scale=0.25)
+    tol = 1e-5 if w.dtype == "f32" else 1e-2
+    assert_parity(np64(xg), ref, max_rel=tol, mean_abs=1e-3 if w.dtype != "f32" else 1e-6, what="rope PI")
+    a, b = x[:, :w.N].cuda(), x[:, :w.N].cuda()  # one frame
+    r.t_scale = 0.5
+    swa.rope_apply(a, 14, r)
+    swa.rope_apply(b, 7, rope_of(w))
+    assert torch.equal(a, b)
+
+
 # ---------------------------------------------------------------------------- append
 @pytest.mark.parametrize("name,chunk", [("tiny", 1), ("chunk", 3)])
 def test_append_slots_and_values(name, chunk):
@@ -125,7 +147,8 @@ def test_append_fp8_codes_and_scales():
 
 # ---------------------------------------------------------------------------- attention
 def run_stream(w: W.Workload, frames, layer=0, rows_per_step=48, q_scale=1.0, check_lse=True, dtype=None,
-               B=None, mean_abs=1e-3, lse_rel=1e-3, max_rel=1e-2, scale=None, k_scale=None, no_rope=False):
+               B=None, mean_abs=1e-3, lse_rel=1e-3, max_rel=1e-2, scale=None, k_scale=None, no_rope=False,
+               t_scale=1.0):
     """Append + attend frame by frame (or chunk by chunk); compare sampled rows
     (all rows when the step is small) with the oracle stream."""
     B = B or w.B
@@ -133,8 +156,11 @@ def run_stream(w: W.Workload, frames, layer=0, rows_per_step=48, q_scale=1.0, ch
     # no_rope: Q and K are passed as already rotated (rope descriptor NULL);
     # the oracle then rotates by angle 0 (all frequencies zero)
     rope = None if no_rope else rope_of(w)
+    if rope is not None:
+        rope.t_scale = t_scale
     om = np.zeros_like(omega_of(w)) if no_rope else omega_of(w)
-    oracles = [StreamOracle(w.H, w.D, w.grid_h, w.grid_w, om, w.pairs, w.t_offset) for _ in range(B)]
+    oracles = [StreamOracle(w.H, w.D, w.grid_h, w.grid_w, om, w.pairs, w.t_offset, t_scale=t_scale)
+               for _ in range(B)]
     c = w.query_frames
     worst = (0.0, 0.0)
     for f0 in frames:
@@ -210,6 +236,30 @@ def test_attention_wan_growing_logits():
     the bar allows for a softmax this sharp."""
     w = W.WAN
     run_stream(w, range(5), rows_per_step=24, q_scale=4.0, k_scale=lambda f: 1.0 + f, no_rope=True)
+
+
+def test_attention_chunk_position_interpolation():
+    """3-frame chunks with jitter, temporal offset 2000 and position
+    interpolation 1/8 on Q and K (append and attention)."""
+    run_stream(W.CHUNK, range(0, 18, 3), rows_per_step=24, t_scale=0.125)
+
+
+def test_phase_coherence_matches_oracle():
+    """ll_phase_coherence against the oracle's C_h(D) for the 12 jittered heads
+    of the chunk workload: offsets around 0, far offsets (10^6 frames) and a
+    position-interpolated band; fp64 on both sides, fp32 output."""
+    w = W.CHUNK
+    om = omega_of(w)
+    pt = w.pairs[0]
+    for delta0, n, ts in [(-64, 4096, 1.0), (10**6, 512, 1.0), (-64, 2048, 0.25)]:
+        r = rope_of(w)
+        r.t_scale = ts
+        got = swa.phase_coherence(r, w.H, delta0, n).cpu().numpy().astype(np.float64)
+        d = np.arange(delta0, delta0 + n, dtype=np.float64) * ts
+        for h in range(w.H):
+            ref = orope.phase_coherence(om[h, :pt], d)
+            err = np.abs(got[h, :, 0] + 1j * got[h, :, 1] - ref)
+            assert err.max() <= 1e-6, (h, delta0, err.max())
 
 
 def test_attention_chunk_jitter():
