@@ -276,6 +276,13 @@ def test_attention_fp8_cache(name, frames):
     run_stream(w, frames, dtype="fp8", rows_per_step=24, mean_abs=5e-3, lse_rel=5e-3, max_rel=5e-2)
 
 
+def test_attention_fp8_cache_d64_staged():
+    """E4M3 cache at D = 64 (dequantised into a bf16 staging copy, then the
+    bf16 kernel): tiny grid, every output row checked."""
+    w = W.replace(W.TINY, dtype="bf16", name="tiny_fp8")
+    run_stream(w, range(14), dtype="fp8", mean_abs=5e-3, lse_rel=5e-3, max_rel=5e-2)
+
+
 def test_attention_chunk_d64_batch3():
     """3-frame chunks at D = 64 (bf16), three independent streams in one call,
     jitter and a temporal offset: 180 query rows per chunk (a full and a
