@@ -32,10 +32,10 @@ def np64(t):
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def setup(w, switch_frame, layer=0, dtype="bf16"):
+def setup(w, switch_frame, layer=0, dtype="bf16", t_scale=1.0):
     eps = W.jitter_eps(11, w.H)
     rope = swa.Rope(pairs=w.pairs, grid_h=w.grid_h, grid_w=w.grid_w, theta0=w.theta0, sigma_t=0.8,
-                    eps=[float(e) for e in eps], t_offset=w.t_offset)
+                    eps=[float(e) for e in eps], t_offset=w.t_offset, t_scale=t_scale)
     om = orope.head_frequencies(w.H, w.pairs, w.theta0, 0.8, eps.astype(np.float64))
     frames = owin.slot_frames(switch_frame - 1)
     n_slots = sum(1 for f in frames if f >= 0)
@@ -47,14 +47,14 @@ def setup(w, switch_frame, layer=0, dtype="bf16"):
     return rope, om, frames[:n_slots], x, wk, wv, gamma, cache
 
 
-def check_slots(w, om, frames, x, wk, wv, gamma, cache, rows_per_slot=None, fp8=False):
+def check_slots(w, om, frames, x, wk, wv, gamma, cache, rows_per_slot=None, fp8=False, t_scale=1.0):
     X, Wk, Wv, G = np64(x[0]), np64(wk), np64(wv), np64(gamma)
     N = w.N
     for s, f in enumerate(frames):
         if rows_per_slot is None:
             rows = np.arange(N)
             kref, vref = orec.recache_frame(X[s * N:(s + 1) * N], Wk, Wv, G, EPS, f, w.H, w.D, w.grid_h, w.grid_w,
-                                            om, w.pairs, w.t_offset)
+                                            om, w.pairs, w.t_offset, t_scale)
         else:
             rows = np.unique(np.r_[0, N - 1, np.random.default_rng(s).choice(N, rows_per_slot, replace=False)])
             kref, vref = _rows_ref(X, Wk, Wv, G, s, f, rows, w, om)
@@ -107,6 +107,14 @@ def test_recache_small_warmup_slots():
     rope, om, frames, x, wk, wv, gamma, cache = setup(w, 7)
     assert len(frames) == 7
     check_slots(w, om, frames, x, wk, wv, gamma, cache)
+
+
+def test_recache_small_position_interpolation():
+    """Position interpolation (t_scale 1/4, temporal offset 300) in the
+    recache epilogue's RoPE; every element checked."""
+    w = W.replace(SMALL, H=4, t_offset=300)
+    rope, om, frames, x, wk, wv, gamma, cache = setup(w, 40, t_scale=0.25)
+    check_slots(w, om, frames, x, wk, wv, gamma, cache, t_scale=0.25)
 
 
 def test_recache_small_fp8():
