@@ -148,19 +148,19 @@ def test_append_fp8_codes_and_scales():
 # ---------------------------------------------------------------------------- attention
 def run_stream(w: W.Workload, frames, layer=0, rows_per_step=48, q_scale=1.0, check_lse=True, dtype=None,
                B=None, mean_abs=1e-3, lse_rel=1e-3, max_rel=1e-2, scale=None, k_scale=None, no_rope=False,
-               t_scale=1.0, lse_mean=5e-3):
+               t_scale=1.0, lse_mean=5e-3, n_sink=3, n_local=9):
     """Append + attend frame by frame (or chunk by chunk); compare sampled rows
     (all rows when the step is small) with the oracle stream."""
     B = B or w.B
-    cache = swa.KVCache(B, w.H, w.D, w.N, dtype or w.dtype)
+    cache = swa.KVCache(B, w.H, w.D, w.N, dtype or w.dtype, n_sink=n_sink, n_local=n_local)
     # no_rope: Q and K are passed as already rotated (rope descriptor NULL);
     # the oracle then rotates by angle 0 (all frequencies zero)
     rope = None if no_rope else rope_of(w)
     if rope is not None:
         rope.t_scale = t_scale
     om = np.zeros_like(omega_of(w)) if no_rope else omega_of(w)
-    oracles = [StreamOracle(w.H, w.D, w.grid_h, w.grid_w, om, w.pairs, w.t_offset, t_scale=t_scale)
-               for _ in range(B)]
+    oracles = [StreamOracle(w.H, w.D, w.grid_h, w.grid_w, om, w.pairs, w.t_offset, t_scale=t_scale,
+                            n_sink=n_sink, n_local=n_local) for _ in range(B)]
     c = w.query_frames
     worst = (0.0, 0.0)
     for f0 in frames:
@@ -211,6 +211,24 @@ def test_attention_tiny_bf16_and_peaked():
 def test_attention_tiny_d128_batch2():
     w = W.replace(W.TINY, dtype="bf16", D=128, pairs=(22, 21, 21), name="tiny_d128")
     run_stream(w, range(14), B=2)
+
+
+@pytest.mark.parametrize("n_sink,n_local", [(0, 5), (1, 1), (4, 12)])
+def test_attention_other_windows(n_sink, n_local):
+    """Other cache shapes: a pure sliding window without sinks, one sink plus
+    only the current frame, and a longer window; 20 frames through warm-up
+    and several ring wraps, every output element checked."""
+    w = W.replace(W.TINY, dtype="bf16", D=128, pairs=(22, 21, 21), name=f"tiny_w{n_sink}_{n_local}")
+    run_stream(w, range(20), n_sink=n_sink, n_local=n_local)
+
+
+def test_attention_max_heads():
+    """H = 64 (the largest head count the descriptors carry), with jitter on
+    every head; every output element checked. The tiny inputs have unit
+    variance, so the logits have unit scale (the Wan frame's 0.25): the LSE
+    bar is the sharper-softmax one (2e-3 of its largest magnitude)."""
+    w = W.replace(W.TINY, dtype="bf16", H=64, name="tiny_h64", sigma_t=0.8, jitter_seed=9)
+    run_stream(w, range(6), lse_rel=2e-3)
 
 
 def test_attention_wan_warmup_and_steady():
