@@ -496,11 +496,12 @@ ll_status ll_append_and_attend(const ll_kvcache* cache, const void* k, const voi
     return fail(LL_ERR_UNSUPPORTED, "tensor too large for one call (%lld items)", ll::append_items(ap));
   // the append's frequency tables are built in the kernel's K stages
   const size_t tables = ll::append_smem_bytes(n_frames, cache->H, cache->D, ap.rp.pt);
-  const size_t kstages = cache->D == 128 ? ll::AttnTraits<128, __nv_bfloat16>::KST * ll::AttnTraits<128, __nv_bfloat16>::KV_BYTES
-                                         : (f32 ? ll::AttnTraits<64, float>::KST * ll::AttnTraits<64, float>::KV_BYTES
-                                                : ll::AttnTraits<64, __nv_bfloat16>::KST * ll::AttnTraits<64, __nv_bfloat16>::KV_BYTES);
-  if (tables > kstages)
-    return fail(LL_ERR_UNSUPPORTED, "frequency tables of %zu bytes exceed %zu", tables, kstages);
+  // the tables live in the kernel's second Q buffer during the append
+  const size_t qbuf = cache->D == 128 ? ll::AttnTraits<128, __nv_bfloat16>::Q_BYTES
+                                      : (f32 ? ll::AttnTraits<64, float>::Q_BYTES
+                                             : ll::AttnTraits<64, __nv_bfloat16>::Q_BYTES);
+  if (tables > qbuf)
+    return fail(LL_ERR_UNSUPPORTED, "frequency tables of %zu bytes exceed %zu", tables, qbuf);
   // the attention part, exactly as ll_sink_window_attention sets it up
   const long long S = cache->n_sink + cache->n_local;
   const long long last = first_frame + n_frames - 1;

@@ -206,7 +206,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* merged = b_ready + 1;     // warpgroup A has read O_A, O_B of the piece
   uint64_t* drain = merged + 1;
   uint64_t* q_tma = drain + 1;        // [2] TMA copy of a Q tile landed
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(q_tma + 2);
+  uint64_t* ap_bar = q_tma + 2;       // fused append: this CTA's K/V rows landed in shared memory
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(ap_bar + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   volatile int* s_last = reinterpret_cast<volatile int*>(s_tmem + 2);
   float* s_mB = reinterpret_cast<float*>(ctrl + 384);      // [128]
@@ -239,6 +240,7 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(drain, 1);
     mbar_init(&q_tma[0], 1);
     mbar_init(&q_tma[1], 1);
+    mbar_init(ap_bar, 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -272,21 +274,85 @@ __global__ void __launch_bounds__(384, 1)
     next_piece(it0, pc0);
     if (threadIdx.x == 64) tma_q_tile<TR>(sQ, &tmQ, &q_tma[0], p, pc0.u);
     if (p.fuse_append) {
-      // the append's tables live in the K stages, which TMA fills only after the barrier
-      float* s_aom = reinterpret_cast<float*>(sK);
-      float* s_atc = s_aom + p.ap.H * (p.ap.D / 2);
-      if (p.ap.rp.enabled) build_append_tables(s_aom, s_atc, p.ap);
-      const long long items = append_items(p.ap);
-      const long long b0 = g * items / p.grid, b1 = (g + 1) * items / p.grid;
-      for (long long i = b0 + threadIdx.x; i < b1; i += blockDim.x) {
-        const AppendItem ai = append_item(p.ap, static_cast<int>(i));
-        float kx[kAppendMaxHg][8], vx[kAppendMaxHg][8];
-        append_load<T>(p.ap, ai, true, kx, vx);
-        if (p.ap.rp.enabled) append_rotate(p.ap, ai, s_aom, s_atc, kx);
-        append_store_plain<T>(p.ap, ai, kx, vx);
+      // This CTA's contiguous share of the new frames' tokens (all batch
+      // entries): their K and V rows come into the K/V stage buffers (which
+      // TMA fills only after the barrier) by bulk copies, K is rotated in
+      // shared memory, and bulk stores write both into the frames' cache
+      // slots. The frequency tables live in the second Q buffer, which the Q
+      // loader fills only after this prologue.
+      const AppendParams& ap = p.ap;
+      float* s_aom = reinterpret_cast<float*>(sQ + TR::Q_BYTES);
+      float* s_atc = s_aom + ap.H * (ap.D / 2);
+      const int RB = ap.H * ap.D * static_cast<int>(sizeof(T));  // bytes of one token row
+      const int FN = ap.F * ap.N, S = ap.n_sink + ap.n_local;
+      const int ttot = ap.B * FN;
+      const int t0 = static_cast<int>(static_cast<long long>(g) * ttot / p.grid);
+      const int t1 = static_cast<int>(static_cast<long long>(g + 1) * ttot / p.grid);
+      const int R = (KST + VST) * TR::KV_BYTES / (2 * RB);  // tokens per round (K half, then V half)
+      uint8_t* sKr = sK;                                     // [R][H][D] K rows
+      uint8_t* sVr = sK + static_cast<size_t>(R) * RB;      // [R][H][D] V rows
+      const T* kin = static_cast<const T*>(ap.k_in);
+      const T* vin = static_cast<const T*>(ap.v_in);
+      T* kc = static_cast<T*>(ap.k_cache);
+      T* vc = static_cast<T*>(ap.v_cache);
+      // the pieces of [r0, r0 + n) that are contiguous in the cache: one (batch, frame) each
+      auto for_segments = [&](int r0, int n, auto&& fn) {
+        for (int r = r0; r < r0 + n;) {
+          const int b = r / FN, rem = r - b * FN, fi = rem / ap.N, nn = rem - fi * ap.N;
+          const int len = min(ap.N - nn, r0 + n - r);
+          const long long crow = (static_cast<long long>(b) * S + cache_slot(ap.first_frame + fi, ap.n_sink,
+                                                                             ap.n_local)) * ap.N + nn;
+          fn(r - r0, static_cast<long long>(r), crow, len);
+          r += len;
+        }
+      };
+      int round = 0;
+      for (int r0 = t0; r0 < t1; r0 += R, ++round) {
+        const int n = min(R, t1 - r0);
+        if (threadIdx.x == 0) {
+          mbar_expect_tx(ap_bar, 2u * static_cast<uint32_t>(n) * RB);
+          bulk_load(sKr, kin + static_cast<size_t>(r0) * ap.H * ap.D, static_cast<uint32_t>(n) * RB, ap_bar);
+          bulk_load(sVr, vin + static_cast<size_t>(r0) * ap.H * ap.D, static_cast<uint32_t>(n) * RB, ap_bar);
+        }
+        if (round == 0 && ap.rp.enabled) build_append_tables(s_aom, s_atc, ap);  // while the rows are in flight
+        const bool landed = mbar_wait(ap_bar, round & 1, s_abort);
+        if (landed && ap.rp.enabled) {
+          const int hg = append_heads_per_thread(ap.H), cpr = ap.D / 8, per_tok = (ap.H / hg) * cpr;
+          for (int i = threadIdx.x; i < n * per_tok; i += blockDim.x) {
+            const int tl = i / per_tok, rem = i - tl * per_tok;
+            const int grp = rem / cpr;
+            const int tg = (r0 + tl) % FN;  // token within the batch entry's new frames
+            AppendItem ai;
+            ai.c = rem - grp * cpr;
+            ai.h0 = grp * hg;
+            ai.fi = tg / ap.N;
+            ai.n = tg - ai.fi * ap.N;
+            T* row = reinterpret_cast<T*>(sKr + static_cast<size_t>(tl) * RB);
+            float kx[kAppendMaxHg][8];
+#pragma unroll
+            for (int k = 0; k < kAppendMaxHg; ++k)
+              if (k < hg) load_chunk8<T>(row + (ai.h0 + k) * ap.D + ai.c * 8, kx[k]);
+            append_rotate(ap, ai, s_aom, s_atc, kx);
+#pragma unroll
+            for (int k = 0; k < kAppendMaxHg; ++k)
+              if (k < hg) store_chunk8<T>(row + (ai.h0 + k) * ap.D + ai.c * 8, kx[k]);
+          }
+        }
+        if (!landed && threadIdx.x == 0) mbar_wait_teardown(ap_bar, round & 1);  // the copies must land
+        fence_proxy_async_smem();  // the rotated rows are read by the bulk stores (async proxy)
+        __syncthreads();
+        if (threadIdx.x == 0) {
+          if (landed)
+            for_segments(r0, n, [&](int off, long long, long long crow, int len) {
+              bulk_store(kc + crow * ap.H * ap.D, sKr + static_cast<size_t>(off) * RB, static_cast<uint32_t>(len) * RB);
+              bulk_store(vc + crow * ap.H * ap.D, sVr + static_cast<size_t>(off) * RB, static_cast<uint32_t>(len) * RB);
+            });
+          bulk_store_commit_wait();  // complete before the rows are reused or the barrier is passed
+        }
+        __syncthreads();
       }
       // the cache rows written here are read by TMA (async proxy) after the
-      // barrier, and TMA refills the K stages that held the tables
+      // barrier, and TMA refills the buffers that held the rows and tables
       asm volatile("fence.proxy.async.global;" ::: "memory");
       fence_proxy_async_smem();
       __threadfence();
