@@ -237,6 +237,19 @@ ll_status ll_phase_coherence(const ll_rope_desc* rope, int H, long long delta0, 
                              void* stream);
 
 /*
+ * Self-test of the library's failure detection (not a step of the method):
+ * every device-side wait in the kernels is bounded, and one that gives up
+ * records LL_ERR_TIMEOUT in the device error word instead of hanging the
+ * context. This launches one CTA that waits on a barrier nothing completes
+ * and on a two-CTA grid barrier that only it reaches; each wait gives up
+ * after the library's bound (about one second of SM clocks) and the kernel
+ * returns. Afterwards ll_device_error() reports LL_ERR_TIMEOUT (and clears
+ * the word) and the context stays usable. Asynchronous on `stream`; the
+ * error word is shared by all calls of the process, so run it alone.
+ */
+ll_status ll_selftest_bounded_waits(void* stream);
+
+/*
  * Allocation-free variant of ll_sink_window_attention (the pages have no
  * counterpart; this is a library convenience).
  * Some callers cannot call cudaMalloc or any allocating routine: cudaMalloc

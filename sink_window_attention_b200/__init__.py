@@ -28,6 +28,7 @@ EXPORTED = (
     "ll_kvcache_append", "ll_sink_window_attention_workspace_bytes", "ll_sink_window_attention",
     "ll_kv_recache_workspace_bytes", "ll_kv_recache", "ll_sink_window_attention_noalloc",
     "ll_append_and_attend_workspace_bytes", "ll_append_and_attend", "ll_phase_coherence",
+    "ll_selftest_bounded_waits",
 )
 NOALLOC_SCRATCH_BYTES = 48 * 1024 * 1024
 
@@ -81,6 +82,7 @@ def lib() -> ctypes.CDLL:
         L.ll_append_and_attend_workspace_bytes.restype = sz
         L.ll_append_and_attend.argtypes = [cp, vp, vp, vp, i, ll_, i, rp, f, vp, vp, vp, sz, vp]
         L.ll_phase_coherence.argtypes = [rp, i, ll_, i, vp, vp]
+        L.ll_selftest_bounded_waits.argtypes = [vp]
         for name in EXPORTED[2:]:
             if not name.endswith("_workspace_bytes"):
                 getattr(L, name).restype = i
@@ -331,3 +333,10 @@ def phase_coherence(rope: Rope, H: int, delta0: int, n_delta: int, out: Optional
     _check(lib().ll_phase_coherence(ctypes.byref(rope.to_c()), H, int(delta0), int(n_delta), _ptr(out),
                                     _stream(stream)))
     return out
+
+
+def selftest_bounded_waits(stream=None) -> int:
+    """Launch the bounded-wait self-test (ll_selftest_bounded_waits) and return
+    the device error code it leaves (read and cleared by ll_device_error)."""
+    _check(lib().ll_selftest_bounded_waits(_stream(stream)))
+    return device_error(stream)

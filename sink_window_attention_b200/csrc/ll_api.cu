@@ -556,6 +556,12 @@ ll_status ll_phase_coherence(const ll_rope_desc* rope, int H, long long delta0, 
   return check_launch("phase_coherence_kernel");
 }
 
+ll_status ll_selftest_bounded_waits(void* stream) {
+  g_last_error.clear();
+  ll::selftest_bounded_waits_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(next_generation());
+  return check_launch("selftest_bounded_waits_kernel");
+}
+
 }  // extern "C"
 
 // Scratch of ll_sink_window_attention_noalloc: one copy per device that loads

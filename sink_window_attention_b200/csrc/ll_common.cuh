@@ -141,6 +141,24 @@ __device__ __forceinline__ bool grid_barrier(unsigned long long* word, unsigned 
   }
 }
 
+// Self-test of the bounded waits: one CTA waits on an mbarrier that nothing
+// completes, then (reset abort flag) on a grid barrier of two CTAs that only
+// it reaches. Both waits give up after kWaitLimitCycles and record
+// kErrWaitTimeout in the error word; the kernel then returns normally.
+__device__ unsigned long long g_selftest_barrier;
+__global__ void selftest_bounded_waits_kernel(unsigned int gen) {
+  __shared__ uint64_t bar;
+  __shared__ volatile int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    mbar_wait(&bar, 0, &abort_flag);  // no arrival ever comes
+    abort_flag = 0;
+    grid_barrier(&g_selftest_barrier, gen, 2u, &abort_flag);  // one of two arrivals
+  }
+}
+
 // Bounded wait used during teardown after an abort: ignores the abort flag.
 __device__ __forceinline__ bool mbar_wait_teardown(uint64_t* bar, uint32_t parity) {
   const uint32_t a = smem_addr(bar);
