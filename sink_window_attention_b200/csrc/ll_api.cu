@@ -106,15 +106,36 @@ ll_status check_grid(const ll_rope_desc* r, int N) {
   return LL_OK;
 }
 
+constexpr int kDeviceSlots = 64;  // device ordinals with cached per-device state
+
+// SM count of the current device (looked up once per device).
 int num_sms() {
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
+  static std::atomic<int> cached[kDeviceSlots];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) dev = 0;
+  if (dev < kDeviceSlots) {
+    const int c = cached[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
   }
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
+  if (dev < kDeviceSlots) cached[dev].store(sms, std::memory_order_relaxed);
   return sms;
+}
+
+// Runs `setup` (kernel attributes: they are per device) the first time it is
+// reached on the current device; later calls on that device skip it. Only a
+// successful setup is remembered.
+template <class F>
+ll_status once_per_device(std::atomic<unsigned long long>& done, F&& setup) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return check_launch("cudaGetDevice");
+  if (dev < 0 || dev >= kDeviceSlots) return fail(LL_ERR_UNSUPPORTED, "device ordinal %d is out of range", dev);
+  const unsigned long long bit = 1ull << dev;
+  if (done.load(std::memory_order_acquire) & bit) return LL_OK;
+  const ll_status st = setup();
+  if (st == LL_OK) done.fetch_or(bit, std::memory_order_acq_rel);
+  return st;
 }
 
 // ---------------------------------------------------------------------------
@@ -191,12 +212,13 @@ ll_status launch_attention(ll::AttnParams p, const ll_kvcache* c, long long S, v
                        TR::ES == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B);
   if (st != LL_OK) return st;
   auto kern = ll::sink_window_attention_kernel<TR>;
-  static bool attr_set = false;
-  if (!attr_set) {
+  static std::atomic<unsigned long long> attr_set{0};
+  st = once_per_device(attr_set, [&]() -> ll_status {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TR::SMEM_BYTES) != cudaSuccess)
       return check_launch("cudaFuncSetAttribute(attention)");
-    attr_set = true;
-  }
+    return LL_OK;
+  });
+  if (st != LL_OK) return st;
   if (cudaMemsetAsync(p.counters, 0, p.units * sizeof(int), stream) != cudaSuccess)
     return check_launch("cudaMemsetAsync(attention counters)");
   if (!cooperative) {
@@ -570,7 +592,7 @@ ll_status ll_selftest_bounded_waits(void* stream) {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[LL_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-constexpr int kMaxDevices = 64;
+constexpr int kMaxDevices = kDeviceSlots;
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kMaxDevices] = {};
 
@@ -687,15 +709,16 @@ ll_status ll_kv_recache(const ll_kvcache* cache, const void* x, int d_model, con
            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return fail(LL_ERR_CUDA, "cuTensorMapEncodeTiled(w) failed");
   }
-  static bool attr_set = false;
-  if (!attr_set) {
+  static std::atomic<unsigned long long> attr_set{0};
+  const ll_status ast = once_per_device(attr_set, []() -> ll_status {
     if (cudaFuncSetAttribute(ll::kv_recache_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TR::SMEM_BYTES) !=
         cudaSuccess)
       return check_launch("cudaFuncSetAttribute(recache)");
     if (cudaFuncSetAttribute(ll::kv_recache_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 0) != cudaSuccess)
       return check_launch("cudaFuncSetAttribute(recache cluster)");
-    attr_set = true;
-  }
+    return LL_OK;
+  });
+  if (ast != LL_OK) return ast;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(Dout / TR::BN, (p.M + TR::BM - 1) / TR::BM, 2 * cache->B);
   cfg.blockDim = dim3(TR::THREADS, 1, 1);
