@@ -1,6 +1,7 @@
 // ll_api.cu — host side of libll_swa.so: argument validation, TMA tensor-map
 // encoding and kernel launches behind the C ABI declared in include/ll_api.h.
 // The library allocates no device memory and keeps no state between calls.
+#include <climits>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -58,6 +59,8 @@ ll_status make_rope(const ll_rope_desc* r, int H, int D, long long t_first, ll::
   if (!(r->sigma_t >= 0.0 && r->sigma_t < 1.0))
     return fail(LL_ERR_INVALID_ARG, "rope sigma_t must lie in [0, 1) so every base stays positive");
   if (r->grid_h < 1 || r->grid_w < 1) return fail(LL_ERR_INVALID_ARG, "rope grid must be at least 1x1");
+  if (static_cast<long long>(r->grid_h) * r->grid_w > INT_MAX)
+    return fail(LL_ERR_INVALID_ARG, "rope grid %dx%d has more than 2^31 - 1 tokens", r->grid_h, r->grid_w);
   if (H > ll::kMaxHeads) return fail(LL_ERR_INVALID_ARG, "H = %d exceeds %d", H, ll::kMaxHeads);
   if (r->t_offset < 0) return fail(LL_ERR_INVALID_ARG, "rope t_offset must be >= 0");
   if (!(r->t_scale >= 0.0 && r->t_scale <= 1.0))
@@ -101,7 +104,7 @@ ll_status check_cache(const ll_kvcache* c) {
 }
 
 ll_status check_grid(const ll_rope_desc* r, int N) {
-  if (r && r->grid_h * r->grid_w != N)
+  if (r && static_cast<long long>(r->grid_h) * r->grid_w != N)
     return fail(LL_ERR_INVALID_ARG, "rope grid %dx%d does not match %d tokens per frame", r->grid_h, r->grid_w, N);
   return LL_OK;
 }

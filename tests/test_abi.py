@@ -113,6 +113,11 @@ def test_append_and_rope_validation(L):
     assert L.ll_rope_apply(None, swa.LL_BF16, 1, 1, 12, 128, 0, rc, None) == swa.LL_ERR_INVALID_ARG
     assert L.ll_rope_apply(k, swa.LL_FP8_E4M3, 1, 1, 12, 128, 0, rc, None) == swa.LL_ERR_INVALID_ARG
     assert L.ll_rope_apply(k, swa.LL_BF16, 1, 1, 12, 128, 0, None, None) == swa.LL_ERR_INVALID_ARG
+    # a grid whose token count overflows 32 bits is rejected, not wrapped
+    big = ctypes.byref(_rope(grid_h=65536, grid_w=65536))
+    assert L.ll_rope_apply(k, swa.LL_BF16, 1, 1, 12, 128, 0, big, None) == swa.LL_ERR_INVALID_ARG
+    assert "2^31" in swa.last_error()
+    assert L.ll_kvcache_append(ctypes.byref(c), k, v, swa.LL_BF16, 0, 1, big, slots, None) == swa.LL_ERR_INVALID_ARG
 
 
 def test_recache_validation(L):
