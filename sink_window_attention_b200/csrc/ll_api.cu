@@ -100,6 +100,9 @@ ll_status check_cache(const ll_kvcache* c) {
   }
   if (c->H > ll::kMaxHeads) return fail(LL_ERR_INVALID_ARG, "H = %d exceeds %d", c->H, ll::kMaxHeads);
   if (c->n_sink < 0 || c->n_local < 1) return fail(LL_ERR_INVALID_ARG, "need n_sink >= 0 and n_local >= 1");
+  if ((static_cast<long long>(c->n_sink) + c->n_local) * c->tokens_per_frame > INT_MAX)
+    return fail(LL_ERR_INVALID_ARG, "(n_sink + n_local) x tokens_per_frame = %lld cache rows exceed 2^31 - 1",
+                (static_cast<long long>(c->n_sink) + c->n_local) * c->tokens_per_frame);
   return LL_OK;
 }
 
@@ -415,6 +418,8 @@ ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvc
   const long long last = first_frame + n_query_frames - 1;
   const long long valid_slots = last + 1 < S ? last + 1 : S;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ll::AttnParams p{};
+  if ((st = make_rope(rope, cache->H, cache->D, first_frame, &p.rp)) != LL_OK) return st;  // before any launch
   ll_kvcache staged;
   if (cache->dtype == LL_FP8_E4M3) {
     // E4M3 cache: the occupied rows are dequantised into bf16 staging inside
@@ -447,8 +452,6 @@ ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvc
     staged.dtype = LL_BF16;
     cache = &staged;
   }
-  ll::AttnParams p{};
-  if ((st = make_rope(rope, cache->H, cache->D, first_frame, &p.rp)) != LL_OK) return st;
   p.q = q;
   p.out = out;
   p.lse = lse;

@@ -72,28 +72,37 @@ def _attn(L, cache, rope=None, first=0, nq=1, scale=0.0, ws=None, ws_bytes=0, q=
 
 
 def test_attention_validation(L):
+    """Every case fails its own check (the workspace is large enough, so the
+    error cannot come from the workspace check), before anything launches."""
+    ws = dict(ws=1 << 24, ws_bytes=1 << 40)
+    fp8 = dict(dtype=swa.LL_FP8_E4M3, k_scale=1 << 22, v_scale=1 << 23)
     bad = [
-        dict(cache=_cache(k=None)),
-        dict(cache=_cache(D=100)),
-        dict(cache=_cache(H=65)),
-        dict(cache=_cache(n_local=0)),
-        dict(cache=_cache(dtype=swa.LL_FP8_E4M3)),            # FP8 without scales
-        dict(cache=_cache(), first=-1),
-        dict(cache=_cache(), nq=0),
-        dict(cache=_cache(), nq=10),
-        dict(cache=_cache(), scale=-1.0),
-        dict(cache=_cache(), q=None),
-        dict(cache=_cache(), q=(1 << 20) + 2),                 # misaligned
-        dict(cache=_cache(), qdt=swa.LL_F32),
-        dict(cache=_cache(), rope=_rope(pairs_t=10)),          # pairs do not sum to D/2
-        dict(cache=_cache(), rope=_rope(grid_w=51)),           # grid does not match N
-        dict(cache=_cache(), rope=_rope(theta0=0.5)),
-        dict(cache=_cache(), rope=_rope(sigma_t=1.5)),
+        (dict(cache=_cache(k=None)), "NULL"),
+        (dict(cache=_cache(D=100)), "multiple of 16"),
+        (dict(cache=_cache(H=65)), "exceeds"),
+        (dict(cache=_cache(n_local=0)), "n_local"),
+        (dict(cache=_cache(tokens_per_frame=1 << 28)), "2^31"),     # cache rows overflow 32 bits
+        (dict(cache=_cache(dtype=swa.LL_FP8_E4M3)), "k_scale"),     # FP8 without scales
+        (dict(cache=_cache(), first=-1), "first_frame"),
+        (dict(cache=_cache(), nq=0), "n_query_frames"),
+        (dict(cache=_cache(), nq=10), "n_query_frames"),
+        (dict(cache=_cache(), scale=-1.0), "softmax_scale"),
+        (dict(cache=_cache(), q=None), "non-NULL"),
+        (dict(cache=_cache(), q=(1 << 20) + 2), "aligned"),
+        (dict(cache=_cache(), qdt=swa.LL_F32), "q dtype"),
+        (dict(cache=_cache(), rope=_rope(pairs_t=10)), "sum to D/2"),
+        (dict(cache=_cache(), rope=_rope(grid_w=51)), "does not match"),
+        (dict(cache=_cache(), rope=_rope(theta0=0.5)), "theta0"),
+        (dict(cache=_cache(), rope=_rope(sigma_t=1.5)), "sigma_t"),
+        # an FP8 cache is dequantised by a kernel: a bad rope must be caught first
+        (dict(cache=_cache(**fp8), rope=_rope(pairs_t=10)), "sum to D/2"),
     ]
-    for kw in bad:
-        st = _attn(L, **kw)
-        assert st == swa.LL_ERR_INVALID_ARG, (kw, st)
-        assert swa.last_error() != ""
+    for kw, msg in bad:
+        st = _attn(L, **{**ws, **kw})
+        assert st == swa.LL_ERR_INVALID_ARG, (kw, st, swa.last_error())
+        assert msg in swa.last_error(), (kw, swa.last_error())
+    assert _attn(L, _cache(), ws=1 << 24, ws_bytes=16) == swa.LL_ERR_INVALID_ARG
+    assert "workspace" in swa.last_error()
 
 
 def test_append_and_rope_validation(L):
