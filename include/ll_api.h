@@ -94,9 +94,10 @@ typedef struct ll_rope_desc {
  * One layer's sink + ring KV cache (caller-owned device memory).
  * k, v: [B][S*N][H][D] of `dtype` (F32, BF16 or FP8_E4M3).
  * k_scale, v_scale: [B][S*N][H] fp32 dequantisation scales, FP8 only
- * (value = decode(code) * scale); NULL for the other dtypes.
+ * (value = decode(code) * scale; 4-byte aligned); NULL for the other dtypes.
  * D: a multiple of 16; an FP8 cache needs D = 16 * 2^k <= 256
  * (LL_ERR_UNSUPPORTED otherwise). k and v must be 16-byte aligned.
+ * S*N (rows per batch entry) must not exceed 2^31 - 1 (LL_ERR_INVALID_ARG).
  */
 typedef struct ll_kvcache {
   void* k;
@@ -174,7 +175,8 @@ ll_status ll_kvcache_append(const ll_kvcache* cache, const void* k, const void* 
  * (rope NULL: q is already rotated).
  * q, out: [B][n_query_frames*N][H][D]; BF16 for BF16 and FP8 caches, F32 for an
  * F32 cache. softmax_scale 0 means 1/sqrt(D). lse (optional, NULL to skip):
- * [B][H][n_query_frames*N] fp32 natural-log sum of exp of the scaled scores.
+ * [B][H][n_query_frames*N] fp32 natural-log sum of exp of the scaled scores,
+ * 4-byte aligned.
  * workspace: device scratch of at least
  * ll_sink_window_attention_workspace_bytes(...) bytes (NULL allowed when that
  * is 0); its contents need not be initialised and are clobbered.
@@ -285,12 +287,15 @@ ll_status ll_sink_window_attention_noalloc(const void* q, ll_dtype q_dtype, cons
  * (BF16; rows of slot s belong to the frame held in slot s):
  *   K = RoPE(RMSNorm(x Wk; gamma, rms_eps)),  V = x Wv,
  * RMSNorm over the whole H*D-wide row, RoPE at each slot's frame position.
- * wk, wv: [d_model][H*D] BF16 row-major; gamma: [H*D] fp32.
- * slot_frames: HOST array of n_slots absolute frame indices (frame in slot s).
+ * wk, wv: [d_model][H*D] BF16 row-major; gamma: [H*D] fp32, 4-byte aligned.
+ * slot_frames: HOST array of n_slots absolute frame indices (frame in slot s),
+ * each in [0, 2^31 - 1].
  * workspace: device scratch of at least ll_kv_recache_workspace_bytes(...)
  * bytes. The cache may be BF16 or FP8.
- * Errors: LL_ERR_INVALID_ARG for NULL pointers, n_slots outside [1, S],
- * negative frames; LL_ERR_UNSUPPORTED for d_model or H*D not a multiple of 128.
+ * Errors: LL_ERR_INVALID_ARG for NULL or misaligned pointers, n_slots outside
+ * [1, S], frames outside [0, 2^31 - 1]; LL_ERR_UNSUPPORTED for a d_model that
+ * is not a positive multiple of 64, for H*D that is not a multiple of 256 up
+ * to 2048 or D other than 64 or 128, and for an F32 cache.
  */
 size_t ll_kv_recache_workspace_bytes(const ll_kvcache* cache, int d_model, int n_slots);
 

@@ -46,6 +46,7 @@ int element_size(ll_dtype t) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 // Validates a rope descriptor for heads H and head dim D and converts it.
 ll_status make_rope(const ll_rope_desc* r, int H, int D, long long t_first, ll::RopeParams* out) {
@@ -89,6 +90,8 @@ ll_status check_cache(const ll_kvcache* c) {
   if (element_size(c->dtype) == 0) return fail(LL_ERR_INVALID_ARG, "unknown cache dtype %d", (int)c->dtype);
   if (c->dtype == LL_FP8_E4M3 && (c->k_scale == nullptr || c->v_scale == nullptr))
     return fail(LL_ERR_INVALID_ARG, "an FP8 cache needs k_scale and v_scale");
+  if (c->dtype == LL_FP8_E4M3 && (!aligned4(c->k_scale) || !aligned4(c->v_scale)))
+    return fail(LL_ERR_INVALID_ARG, "k_scale and v_scale must be 4-byte aligned");
   if (c->B < 1 || c->H < 1 || c->D < 2 || c->tokens_per_frame < 1)
     return fail(LL_ERR_INVALID_ARG, "cache sizes must be positive (B=%d H=%d D=%d N=%d)", c->B, c->H, c->D,
                 c->tokens_per_frame);
@@ -400,6 +403,7 @@ ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvc
   if (st != LL_OK) return st;
   if (q == nullptr || out == nullptr) return fail(LL_ERR_INVALID_ARG, "q and out must be non-NULL");
   if (!aligned16(q) || !aligned16(out)) return fail(LL_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
+  if (!aligned4(lse)) return fail(LL_ERR_INVALID_ARG, "lse must be 4-byte aligned");
   if (first_frame < 0) return fail(LL_ERR_INVALID_ARG, "first_frame must be >= 0");
   if (n_query_frames < 1 || n_query_frames > cache->n_local)
     return fail(LL_ERR_INVALID_ARG, "n_query_frames = %d must lie in [1, n_local = %d]", n_query_frames,
@@ -491,6 +495,7 @@ ll_status ll_append_and_attend(const ll_kvcache* cache, const void* k, const voi
     return fail(LL_ERR_INVALID_ARG, "k, v, q and out must be non-NULL");
   if (!aligned16(k) || !aligned16(v) || !aligned16(q) || !aligned16(out))
     return fail(LL_ERR_INVALID_ARG, "k, v, q and out must be 16-byte aligned");
+  if (!aligned4(lse)) return fail(LL_ERR_INVALID_ARG, "lse must be 4-byte aligned");
   if (first_frame < 0) return fail(LL_ERR_INVALID_ARG, "first_frame must be >= 0");
   if (n_frames < 1 || n_frames > cache->n_local)
     return fail(LL_ERR_INVALID_ARG, "n_frames = %d must lie in [1, n_local = %d]", n_frames, cache->n_local);
@@ -660,11 +665,13 @@ ll_status ll_kv_recache(const ll_kvcache* cache, const void* x, int d_model, con
     return fail(LL_ERR_INVALID_ARG, "x, wk, wv, gamma and slot_frames must be non-NULL");
   if (!aligned16(x) || !aligned16(wk) || !aligned16(wv))
     return fail(LL_ERR_INVALID_ARG, "x, wk and wv must be 16-byte aligned");
+  if (!aligned4(gamma)) return fail(LL_ERR_INVALID_ARG, "gamma must be 4-byte aligned");
   const int S = cache->n_sink + cache->n_local;
   if (n_slots < 1 || n_slots > S || n_slots > ll::kMaxSlots)
     return fail(LL_ERR_INVALID_ARG, "n_slots = %d must lie in [1, %d]", n_slots, S < ll::kMaxSlots ? S : ll::kMaxSlots);
   for (int i = 0; i < n_slots; ++i)
-    if (slot_frames[i] < 0) return fail(LL_ERR_INVALID_ARG, "slot_frames[%d] is negative", i);
+    if (slot_frames[i] < 0 || slot_frames[i] > INT_MAX)
+      return fail(LL_ERR_INVALID_ARG, "slot_frames[%d] = %lld lies outside [0, 2^31 - 1]", i, slot_frames[i]);
   if (!(rms_eps >= 0.f) || !std::isfinite(rms_eps)) return fail(LL_ERR_INVALID_ARG, "rms_eps must be finite, >= 0");
   if ((st = check_grid(rope, cache->tokens_per_frame)) != LL_OK) return st;
   if (cache->dtype != LL_BF16 && cache->dtype != LL_FP8_E4M3)

@@ -65,9 +65,9 @@ def _rope(**kw):
 
 
 def _attn(L, cache, rope=None, first=0, nq=1, scale=0.0, ws=None, ws_bytes=0, q=1 << 20, out=1 << 21,
-          qdt=swa.LL_BF16):
+          qdt=swa.LL_BF16, lse=None):
     return L.ll_sink_window_attention(q, qdt, ctypes.byref(cache), first, nq,
-                                      ctypes.byref(rope) if rope is not None else None, scale, out, None, ws,
+                                      ctypes.byref(rope) if rope is not None else None, scale, out, lse, ws,
                                       ws_bytes, None)
 
 
@@ -90,6 +90,7 @@ def test_attention_validation(L):
         (dict(cache=_cache(), q=None), "non-NULL"),
         (dict(cache=_cache(), q=(1 << 20) + 2), "aligned"),
         (dict(cache=_cache(), qdt=swa.LL_F32), "q dtype"),
+        (dict(cache=_cache(), lse=(1 << 25) + 2), "lse"),
         (dict(cache=_cache(), rope=_rope(pairs_t=10)), "sum to D/2"),
         (dict(cache=_cache(), rope=_rope(grid_w=51)), "does not match"),
         (dict(cache=_cache(), rope=_rope(theta0=0.5)), "theta0"),
@@ -133,8 +134,8 @@ def test_recache_validation(L):
     c = _cache()
     frames = (ctypes.c_longlong * 12)(*range(12))
     g = 1 << 22
-    def call(cache=c, n=12, dm=1536, fr=frames, x=1 << 20):
-        return L.ll_kv_recache(ctypes.byref(cache), x, dm, 1 << 21, 1 << 21, g, 1e-6, fr, n, None, None, 0, None)
+    def call(cache=c, n=12, dm=1536, fr=frames, x=1 << 20, gamma=g):
+        return L.ll_kv_recache(ctypes.byref(cache), x, dm, 1 << 21, 1 << 21, gamma, 1e-6, fr, n, None, None, 0, None)
     assert call(n=0) == swa.LL_ERR_INVALID_ARG
     assert call(n=13) == swa.LL_ERR_INVALID_ARG
     assert call(x=None) == swa.LL_ERR_INVALID_ARG
@@ -142,6 +143,13 @@ def test_recache_validation(L):
     assert call(dm=100) == swa.LL_ERR_UNSUPPORTED
     assert call(cache=_cache(H=3)) == swa.LL_ERR_UNSUPPORTED        # H*D = 384 is not a multiple of 256
     assert call(cache=_cache(dtype=swa.LL_F32)) == swa.LL_ERR_UNSUPPORTED
+    assert call(gamma=g + 2) == swa.LL_ERR_INVALID_ARG                    # gamma read as floats
+    assert "gamma" in swa.last_error()
+    assert call(fr=(ctypes.c_longlong * 12)(*([1 << 40] * 12))) == swa.LL_ERR_INVALID_ARG  # frame beyond 32 bits
+    assert "slot_frames[0]" in swa.last_error()
+    fp8 = _cache(dtype=swa.LL_FP8_E4M3, k_scale=(1 << 22) + 1, v_scale=1 << 23)
+    assert call(cache=fp8) == swa.LL_ERR_INVALID_ARG                      # scales written as floats
+    assert "4-byte" in swa.last_error()
 
 
 def _fused(L, cache, rope=None, first=0, nf=1, scale=0.0, ws=1 << 24, ws_bytes=1 << 30, k=1 << 20, v=1 << 21,
