@@ -114,11 +114,31 @@ def _dtype_code(t: torch.dtype) -> int:
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    """Device address of a contiguous CUDA tensor on the current device (the
+    library's kernels dereference it there)."""
     if t is None:
         return None
+    if not t.is_cuda:
+        raise ValueError(f"tensors must be CUDA tensors, got one on {t.device}")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"tensors must be on the current CUDA device (cuda:{torch.cuda.current_device()}), "
+                         f"got one on {t.device}")
     if not t.is_contiguous():
         raise ValueError("tensors must be contiguous")
     return t.data_ptr()
+
+
+def _expect(t: Optional[torch.Tensor], shape, dtype: torch.dtype, what: str) -> None:
+    """Shape and dtype of a buffer the kernels read or write in full."""
+    if t is not None and (tuple(t.shape) != tuple(shape) or t.dtype != dtype):
+        raise ValueError(f"{what} must be a {dtype} tensor of shape {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+
+
+def _cache_c(cache: "KVCache") -> "KVCacheC":
+    """The cache descriptor for a launch: its tensors checked like any other."""
+    for t in (cache.k, cache.v, cache.k_scale, cache.v_scale):
+        _ptr(t)
+    return cache.to_c()
 
 
 @dataclass
@@ -205,8 +225,12 @@ def device_error(stream=None) -> int:
 
 def rope_apply(x: torch.Tensor, first_frame: int, rope: Rope, stream=None) -> torch.Tensor:
     """In-place 3D RoPE of x [B, F*N, H, D]."""
+    if x.dim() != 4:
+        raise ValueError(f"x must be [B, F*N, H, D], got shape {tuple(x.shape)}")
     B, T, H, D = x.shape
     N = rope.grid_h * rope.grid_w
+    if T % N != 0:
+        raise ValueError(f"x holds {T} tokens, not a whole number of {N}-token frames")
     _check(lib().ll_rope_apply(_ptr(x), _dtype_code(x.dtype), B, T // N, H, D, first_frame, _rope_ref(rope),
                                _stream(stream)))
     return x
@@ -227,8 +251,10 @@ def kvcache_append(cache: KVCache, k: torch.Tensor, v: torch.Tensor, first_frame
     F = _check_shape(cache, k, "k")
     if _check_shape(cache, v, "v") != F:
         raise ValueError("k and v must cover the same frames")
+    if v.dtype != k.dtype:
+        raise ValueError("k and v must have one dtype")
     slots = (ctypes.c_int * F)()
-    _check(lib().ll_kvcache_append(ctypes.byref(cache.to_c()), _ptr(k), _ptr(v), _dtype_code(k.dtype), first_frame,
+    _check(lib().ll_kvcache_append(ctypes.byref(_cache_c(cache)), _ptr(k), _ptr(v), _dtype_code(k.dtype), first_frame,
                                    F, _rope_ref(rope), slots, _stream(stream)))
     return list(slots)
 
@@ -260,10 +286,12 @@ def sink_window_attention(q: torch.Tensor, cache: KVCache, first_frame: int, rop
     F = _check_shape(cache, q, "q")
     if out is None:
         out = torch.empty_like(q)
+    _expect(out, q.shape, q.dtype, "out")
+    _expect(lse, (cache.B, cache.H, q.shape[1]), torch.float32, "lse")
     if workspace is None:
         workspace = workspace_for(attention_workspace_bytes(cache, F), q.device)
     ws_bytes = workspace.numel() * workspace.element_size()
-    _check(lib().ll_sink_window_attention(_ptr(q), _dtype_code(q.dtype), ctypes.byref(cache.to_c()), first_frame, F,
+    _check(lib().ll_sink_window_attention(_ptr(q), _dtype_code(q.dtype), ctypes.byref(_cache_c(cache)), first_frame, F,
                                           _rope_ref(rope), float(softmax_scale), _ptr(out), _ptr(lse),
                                           _ptr(workspace), ws_bytes, _stream(stream)))
     return out
@@ -282,12 +310,16 @@ def append_and_attend(cache: KVCache, k: torch.Tensor, v: torch.Tensor, q: torch
     F = _check_shape(cache, q, "q")
     if _check_shape(cache, k, "k") != F or _check_shape(cache, v, "v") != F:
         raise ValueError("k, v and q must cover the same frames")
+    if not (k.dtype == v.dtype == q.dtype):
+        raise ValueError("k, v and q must have one dtype")
     if out is None:
         out = torch.empty_like(q)
+    _expect(out, q.shape, q.dtype, "out")
+    _expect(lse, (cache.B, cache.H, q.shape[1]), torch.float32, "lse")
     if workspace is None:
         workspace = workspace_for(append_and_attend_workspace_bytes(cache, F), q.device)
     ws_bytes = workspace.numel() * workspace.element_size()
-    _check(lib().ll_append_and_attend(ctypes.byref(cache.to_c()), _ptr(k), _ptr(v), _ptr(q), _dtype_code(q.dtype),
+    _check(lib().ll_append_and_attend(ctypes.byref(_cache_c(cache)), _ptr(k), _ptr(v), _ptr(q), _dtype_code(q.dtype),
                                       first_frame, F, _rope_ref(rope), float(softmax_scale), _ptr(out), _ptr(lse),
                                       _ptr(workspace), ws_bytes, _stream(stream)))
     return out
@@ -301,7 +333,9 @@ def sink_window_attention_noalloc(q: torch.Tensor, cache: KVCache, first_frame: 
     F = _check_shape(cache, q, "q")
     if out is None:
         out = torch.empty_like(q)
-    _check(lib().ll_sink_window_attention_noalloc(_ptr(q), _dtype_code(q.dtype), ctypes.byref(cache.to_c()),
+    _expect(out, q.shape, q.dtype, "out")
+    _expect(lse, (cache.B, cache.H, q.shape[1]), torch.float32, "lse")
+    _check(lib().ll_sink_window_attention_noalloc(_ptr(q), _dtype_code(q.dtype), ctypes.byref(_cache_c(cache)),
                                                   first_frame, F, _rope_ref(rope), float(softmax_scale), _ptr(out),
                                                   _ptr(lse), _stream(stream)))
     return out
@@ -316,9 +350,16 @@ def kv_recache(cache: KVCache, x: torch.Tensor, wk: torch.Tensor, wv: torch.Tens
                workspace: Optional[torch.Tensor] = None, stream=None) -> None:
     """Recompute K/V of slots 0..len(slot_frames)-1 from hidden states x [B, n*N, d_model]."""
     n = len(slot_frames)
+    if x.dim() != 3:
+        raise ValueError(f"x must be [B, n_slots*N, d_model], got shape {tuple(x.shape)}")
+    dm, dout = x.shape[-1], cache.H * cache.D
+    _expect(x, (cache.B, n * cache.N, dm), torch.bfloat16, "x")
+    _expect(wk, (dm, dout), torch.bfloat16, "wk")
+    _expect(wv, (dm, dout), torch.bfloat16, "wv")
+    _expect(gamma, (dout,), torch.float32, "gamma")
     frames = (ctypes.c_longlong * n)(*[int(f) for f in slot_frames])
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib().ll_kv_recache(ctypes.byref(cache.to_c()), _ptr(x), x.shape[-1], _ptr(wk), _ptr(wv), _ptr(gamma),
+    _check(lib().ll_kv_recache(ctypes.byref(_cache_c(cache)), _ptr(x), dm, _ptr(wk), _ptr(wv), _ptr(gamma),
                                float(rms_eps), frames, n, _rope_ref(rope), _ptr(workspace), ws_bytes,
                                _stream(stream)))
 
@@ -330,6 +371,7 @@ def phase_coherence(rope: Rope, H: int, delta0: int, n_delta: int, out: Optional
     current CUDA device."""
     if out is None:
         out = torch.empty((H, n_delta, 2), dtype=torch.float32, device="cuda")
+    _expect(out, (H, n_delta, 2), torch.float32, "out")
     _check(lib().ll_phase_coherence(ctypes.byref(rope.to_c()), H, int(delta0), int(n_delta), _ptr(out),
                                     _stream(stream)))
     return out

@@ -204,3 +204,33 @@ def test_phase_coherence_and_position_interpolation_validation(L):
         assert L.ll_phase_coherence(ctypes.byref(rb), 12, 0, 16, out, None) == swa.LL_ERR_INVALID_ARG
         assert "t_scale" in swa.last_error()
         assert _attn(L, _cache(), rope=rb, ws=1 << 24, ws_bytes=1 << 30) == swa.LL_ERR_INVALID_ARG
+
+
+def test_binding_rejects_host_tensors_and_mismatched_buffers(L):
+    """The Python binding hands the library device addresses only: host tensors,
+    and buffers whose shape or dtype the kernels would overrun, are refused
+    before any call reaches the library."""
+    import torch
+    B, H, D, N = 1, 2, 64, 24
+    cache = swa.KVCache(B, H, D, N, "bf16", device="cpu")
+    rope = swa.Rope(pairs=(12, 10, 10), grid_h=4, grid_w=6)
+    q = torch.zeros(B, N, H, D, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        swa.sink_window_attention(q, cache, 0, rope)
+    with pytest.raises(ValueError, match="lse"):
+        swa.sink_window_attention(q, cache, 0, rope, lse=torch.zeros(B, H, N + 1))
+    with pytest.raises(ValueError, match="out"):
+        swa.sink_window_attention(q, cache, 0, rope, out=torch.zeros(B, N, H, D))   # f32 out for bf16 q
+    with pytest.raises(ValueError, match="one dtype"):
+        swa.kvcache_append(cache, q, q.float(), 0, rope)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        swa.kvcache_append(cache, q, q, 0, rope)
+    dm, dout = 256, H * D
+    x = torch.zeros(B, N, dm, dtype=torch.bfloat16)
+    w = torch.zeros(dm, dout, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="gamma"):
+        swa.kv_recache(cache, x, w, w, torch.ones(dout, dtype=torch.bfloat16), 1e-6, [0], rope)
+    with pytest.raises(ValueError, match="x must be"):
+        swa.kv_recache(cache, x, w, w, torch.ones(dout), 1e-6, [0, 1], rope)                  # 2 slots need 2N rows
+    with pytest.raises(ValueError, match="whole number"):
+        swa.rope_apply(torch.zeros(B, N + 1, H, D, dtype=torch.bfloat16), 0, rope)
