@@ -143,3 +143,43 @@ def test_stream_denoising_passes_match_dense_masked(chunk):
             assert np.allclose(got, ref, rtol=1e-11, atol=1e-11)
     with pytest.raises(AssertionError):  # a pass may only re-write the most recent frames
         so.append(0, K[0][:N], V[0][:N], replace=True)
+
+
+def test_stream_recache_matches_dense_recomputed():
+    """A prompt switch before frame F (LongLive review, 'KV Recache': the cache
+    is rebuilt from the generated frames with the new prompt). Afterwards every
+    frame the next query can see, sinks included, holds K/V recomputed from its
+    own hidden states at its own position; frame F is appended as usual. One
+    dense masked softmax over those K/V, built frame by frame from
+    recache_frame and rope_frames, must equal the stream oracle's attention."""
+    from oracle import recache
+    Wl = W.TINY
+    H, D, gh, gw = Wl.H, Wl.D, Wl.grid_h, Wl.grid_w
+    N, F, dm, t0 = gh * gw, 16, 32, 100
+    om = rope.head_frequencies(H, Wl.pairs, 10000.0, 0.8, W.jitter_eps(6, H))
+    rng = np.random.default_rng(7)
+    K = rng.standard_normal(((F + 1) * N, H, D))
+    V = rng.standard_normal(((F + 1) * N, H, D))
+    so = StreamOracle(H, D, gh, gw, om, Wl.pairs, t_offset=t0)
+    for f in range(F):
+        so.append(f, K[f * N:(f + 1) * N], V[f * N:(f + 1) * N])
+    X = {g: rng.standard_normal((N, dm)) for g in range(F)}
+    wk = rng.standard_normal((dm, H * D)) / np.sqrt(dm)
+    wv = rng.standard_normal((dm, H * D)) / np.sqrt(dm)
+    gamma = rng.uniform(0.5, 1.5, H * D)
+    so.recache(F, X, wk, wv, gamma, 1e-6)
+    so.append(F, K[F * N:], V[F * N:])
+    q = rng.standard_normal((N, H, D))
+    got = so.attend(q, F)
+    keys, vals = [], []
+    for g in range(F):
+        k, v = recache.recache_frame(X[g], wk, wv, gamma, 1e-6, g, H, D, gh, gw, om, Wl.pairs, t_offset=t0)
+        keys.append(k)
+        vals.append(v)
+    keys.append(rope.rope_frames(K[None, F * N:], F, gh, gw, om, Wl.pairs, t0)[0])
+    vals.append(V[F * N:])
+    A = set(window.attended_frames(F, 3, 9))
+    qr = rope.rope_frames(q[None], F, gh, gw, om, Wl.pairs, t0)[0]
+    ref = _dense_masked(qr, np.concatenate(keys), np.concatenate(vals), np.full(N, F),
+                        np.repeat(np.arange(F + 1), N), lambda qf, kf: kf in A, 1 / np.sqrt(D))
+    assert np.allclose(got, ref, rtol=1e-11, atol=1e-11)

@@ -225,6 +225,31 @@ def append_keys_at_their_slot(self, first_frame, k, v, replace=False):
     self.last = first_frame + F - 1
 
 
+def recache_local_frames_only(self, switch_frame, x_by_frame, wk, wv, gamma, eps):
+    frames = [g for g in window.attended_frames(switch_frame - 1, self.n_sink, self.n_local) if g >= self.n_sink]
+    for g in frames:
+        self.k[g], self.v[g] = recache.recache_frame(x_by_frame[g], wk, wv, gamma, eps, g, self.H, self.D,
+                                                     self.grid_h, self.grid_w, self.omega, self.pairs,
+                                                     self.t_offset, self.t_scale)
+
+
+def recache_at_slot_positions(self, switch_frame, x_by_frame, wk, wv, gamma, eps):
+    for g in window.attended_frames(switch_frame - 1, self.n_sink, self.n_local):
+        s = window.slot_of(g, self.n_sink, self.n_local)
+        self.k[g], self.v[g] = recache.recache_frame(x_by_frame[g], wk, wv, gamma, eps, s, self.H, self.D,
+                                                     self.grid_h, self.grid_w, self.omega, self.pairs,
+                                                     self.t_offset, self.t_scale)
+
+
+@pytest.mark.parametrize("wrong", [recache_local_frames_only, recache_at_slot_positions],
+                         ids=["sinks not recomputed", "frames at their slot positions"])
+def test_stream_recache_pin_rejects(wrong, monkeypatch):
+    pin = [pin_att.test_stream_recache_matches_dense_recomputed]
+    assert not rejected(pin)
+    monkeypatch.setattr(StreamOracle, "recache", wrong)
+    assert rejected(pin)
+
+
 def test_stream_pin_rejects_keys_rotated_at_their_slot(monkeypatch):
     """K must turn with its frame's absolute position, not its cache slot."""
     pin = [lambda: pin_att.test_stream_matches_dense_masked_brute_force(9, 1)]
