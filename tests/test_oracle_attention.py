@@ -183,3 +183,33 @@ def test_stream_recache_matches_dense_recomputed():
     ref = _dense_masked(qr, np.concatenate(keys), np.concatenate(vals), np.full(N, F),
                         np.repeat(np.arange(F + 1), N), lambda qf, kf: kf in A, 1 / np.sqrt(D))
     assert np.allclose(got, ref, rtol=1e-11, atol=1e-11)
+
+
+def test_stream_position_interpolation_matches_dense():
+    """With position interpolation (temporal positions scaled by s, LoL review's
+    PI baseline) the stream equals one dense masked softmax over queries and
+    keys rotated by rope_frames at the scaled positions, and differs from the
+    unscaled stream."""
+    Wl = W.TINY
+    H, D, gh, gw = Wl.H, Wl.D, Wl.grid_h, Wl.grid_w
+    N, F, t0, s = gh * gw, 14, 30, 0.5
+    om = rope.head_frequencies(H, Wl.pairs, 10000.0, 0.8, W.jitter_eps(8, H))
+    rng = np.random.default_rng(9)
+    Q = rng.standard_normal((F * N, H, D))
+    K = rng.standard_normal((F * N, H, D))
+    V = rng.standard_normal((F * N, H, D))
+    so = StreamOracle(H, D, gh, gw, om, Wl.pairs, t_offset=t0, t_scale=s)
+    plain = StreamOracle(H, D, gh, gw, om, Wl.pairs, t_offset=t0)
+    Qr = rope.rope_frames(Q[None], 0, gh, gw, om, Wl.pairs, t0, s)[0]
+    Kr = rope.rope_frames(K[None], 0, gh, gw, om, Wl.pairs, t0, s)[0]
+    kframe = np.repeat(np.arange(F), N)
+    for f in range(F):
+        cur = slice(f * N, (f + 1) * N)
+        so.append(f, K[cur], V[cur])
+        plain.append(f, K[cur], V[cur])
+        got = so.attend(Q[cur], f)
+        A = set(window.attended_frames(f, 3, 9))
+        ref = _dense_masked(Qr[cur], Kr, V, np.full(N, f), kframe, lambda qf, kf: kf in A, 1 / np.sqrt(D))
+        assert np.allclose(got, ref, rtol=1e-11, atol=1e-11)
+        if f >= 4:
+            assert not np.allclose(got, plain.attend(Q[cur], f), atol=1e-6)

@@ -250,6 +250,30 @@ def test_stream_recache_pin_rejects(wrong, monkeypatch):
     assert rejected(pin)
 
 
+def append_pass_not_replacing(self, first_frame, k, v, replace=False):
+    if replace:
+        return  # the pass's K/V never reach the cache
+    StreamOracle.__dict__["_append_orig"](self, first_frame, k, v, replace)
+
+
+def rot_ignoring_interpolation(self, x, frame):
+    t, r, c = rope.token_positions(frame, self.grid_h, self.grid_w, self.t_offset)
+    return rope.rope_3d(x, t, r, c, self.omega, self.pairs)
+
+
+def test_stream_pins_reject_lost_denoising_pass_and_lost_interpolation(monkeypatch):
+    passes = [lambda: pin_att.test_stream_denoising_passes_match_dense_masked(1)]
+    pi = [pin_att.test_stream_position_interpolation_matches_dense]
+    assert not rejected(passes) and not rejected(pi)
+    with monkeypatch.context() as m:
+        m.setattr(StreamOracle, "_append_orig", StreamOracle.append, raising=False)
+        m.setattr(StreamOracle, "append", append_pass_not_replacing)
+        assert rejected(passes)
+    with monkeypatch.context() as m:
+        m.setattr(StreamOracle, "_rot", rot_ignoring_interpolation)
+        assert rejected(pi)
+
+
 def test_stream_pin_rejects_keys_rotated_at_their_slot(monkeypatch):
     """K must turn with its frame's absolute position, not its cache slot."""
     pin = [lambda: pin_att.test_stream_matches_dense_masked_brute_force(9, 1)]
