@@ -1,0 +1,68 @@
+"""Host logic of bench.py that needs no GPU: the algorithmic FLOP and byte
+counts behind the roofline, the clock-sample parsing that decides whether a
+run is kept, the frames a recache recomputes, and the DRAM figure taken from
+a committed ncu summary."""
+import types
+
+import bench
+import swa_workloads as W
+import sink_window_attention_b200 as swa
+from oracle import window
+
+
+def test_algorithmic_flops_and_bytes():
+    # softmax(Q K^T) V per head: 2*Nq*Nk*D for Q K^T and as many for P V
+    assert bench.attention_flops(W.WAN) == 4 * 1560 * 18720 * 128 * 12          # 179.4 GFLOP per layer-step
+    assert round(bench.attention_flops(W.WAN) / 1e9, 1) == 179.4
+    assert bench.attention_flops(W.CHUNK) == 4 * 3 * 1560 * 18720 * 128 * 12    # 3-frame chunk: 538.3 GFLOP
+    n = 1560 * 12 * 128
+    # append: read K, V (bf16), write them to the cache; FP8 adds one fp32 scale per (token, head)
+    assert bench.append_bytes(W.WAN, 2) == 8 * n                                 # 19.2 MB
+    assert bench.append_bytes(W.WAN, 1) == 4 * n + 2 * n + 2 * 1560 * 12 * 4
+
+
+def _sampler_with(lines):
+    s = bench.ClockSampler("0")
+    s.proc = types.SimpleNamespace(terminate=lambda: None, wait=lambda timeout=None: 0, kill=lambda: None)
+    s.thread = types.SimpleNamespace(join=lambda timeout=None: None)
+    s.lines = lines
+    return s
+
+
+def test_clock_samples_give_median_and_active_reasons():
+    row = "0, {sm}, 1965, 900.5, 0x{a:x}, {hw}, Not Active, Not Active, {cap}"
+    lines = [row.format(sm=sm, a=4, hw="Not Active", cap="Active") for sm in (1700, 1710, 1720)]
+    lines.append("garbage line")
+    got = _sampler_with(lines).stop()
+    assert got["sm_mhz"] == 1710 and got["sm_max_mhz"] == 1965 and got["samples"] == 3
+    assert got["reasons"] == ["sw_power_cap"]
+    lines.append(row.format(sm=1200, a=8, hw="Active", cap="Not Active"))
+    assert _sampler_with(lines).stop()["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    none = bench.ClockSampler("0").stop()                  # nvidia-smi never started
+    assert none["sm_mhz"] is None and none["reasons"] == ["nvidia-smi unavailable"]
+
+
+def test_recache_recomputes_exactly_the_cached_frames():
+    """At a prompt switch before frame F the recache rebuilds the frames the
+    cache holds after frame F-1 (LongLive review, 'KV Recache'), in slot order."""
+    fake = types.SimpleNamespace(w=W.STREAM, swa=swa)
+    for last in (0, 1, 2, 5, 11, 12, 39, 40, 79, 919):
+        held = bench.Stream.held_frames(fake, last)
+        assert sorted(held) == window.attended_frames(last, 3, 9)
+        assert held == [f for f in window.slot_frames(last, 3, 9) if f >= 0]
+
+
+def test_traffic_figure_only_for_the_captured_kernel(tmp_path, monkeypatch):
+    """The bench line's roofline.traffic comes from a committed ncu summary only
+    while the attention sources hash to the version that summary names;
+    otherwise it is null (a stale DRAM figure is never reported)."""
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "k.md").write_text("kernel_source_sha256_16: 0123456789abcdef\n\n"
+                               "| dram_bytes_per_launch (read + write) | 230756864 |\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0123456789abcdef")
+    assert bench.load_traffic("k.md") == 230756864
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "fedcba9876543210")
+    assert bench.load_traffic("k.md") is None
+    assert bench.load_traffic("missing.md") is None

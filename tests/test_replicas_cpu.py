@@ -66,3 +66,4 @@ def test_replicas_two_ranks_gloo():
 def test_single_process_max_is_identity():
     import bench
     assert bench.max_over_ranks(3.25, False) == 3.25
+
