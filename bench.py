@@ -120,8 +120,7 @@ class ClockSampler:
             for n, v in zip(names, parts[5:9]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
-        # samples under load: the upper half of the clock distribution is
-        # reported as median; idle samples at the edges are dropped
+        # the median over every sample taken while the timed region ran
         med = statistics.median(sm) if sm else None
         return {"sm_mhz": med, "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
 
