@@ -135,8 +135,11 @@ ll_status ll_device_error(int* code, void* stream);
  * In-place 3D RoPE of x [B][n_frames*N][H][D] (dtype F32 or BF16) holding the
  * consecutive frames first_frame .. first_frame + n_frames - 1.
  * LoL review, "Method steps" (6): (Q'_h, K'_h) = RoPERotate(Q_h, K_h, omega_h).
- * Errors: LL_ERR_INVALID_ARG for NULL x or rope, non-positive sizes,
- * first_frame < 0, D odd or pairs not summing to D/2, H > LL_MAX_HEADS.
+ * Errors: LL_ERR_INVALID_ARG for NULL x or rope, x not 16-byte aligned,
+ * non-positive sizes, first_frame < 0, D not a multiple of 8, a dtype other
+ * than F32 / BF16, or an invalid rope descriptor (pairs not summing to D/2,
+ * H > LL_MAX_HEADS, ...); LL_ERR_UNSUPPORTED for 2^31 or more 8-element
+ * chunks in one call.
  */
 ll_status ll_rope_apply(void* x, ll_dtype dtype, int B, int n_frames, int H, int D,
                         long long first_frame, const ll_rope_desc* rope, void* stream);
@@ -154,9 +157,11 @@ ll_status ll_rope_apply(void* x, ll_dtype dtype, int B, int n_frames, int H, int
  * the same slots again (one call per denoising pass of the current frame, the
  * last pass's K/V staying in the cache).
  * slots_out: optional HOST array of n_frames ints receiving the slots written.
- * Errors: LL_ERR_INVALID_ARG for NULL tensors, first_frame < 0,
- * n_frames < 1 or > n_local (a call may not overwrite its own frames),
- * dtype mismatch with the cache, rope grid inconsistent with N.
+ * Errors: LL_ERR_INVALID_ARG for NULL or misaligned tensors (k, v 16-byte
+ * aligned), first_frame < 0, n_frames < 1 or > n_local (a call may not
+ * overwrite its own frames), dtype mismatch with the cache, a rope grid
+ * inconsistent with N or an otherwise invalid rope descriptor, an invalid
+ * cache descriptor.
  */
 ll_status ll_kvcache_append(const ll_kvcache* cache, const void* k, const void* v,
                             ll_dtype in_dtype, long long first_frame, int n_frames,
@@ -180,9 +185,13 @@ ll_status ll_kvcache_append(const ll_kvcache* cache, const void* k, const void* 
  * workspace: device scratch of at least
  * ll_sink_window_attention_workspace_bytes(...) bytes (NULL allowed when that
  * is 0); its contents need not be initialised and are clobbered.
- * Errors: LL_ERR_INVALID_ARG for NULL tensors, first_frame < 0,
- * n_query_frames < 1 or > n_local, a workspace that is too small;
- * LL_ERR_UNSUPPORTED for D other than 64 or 128.
+ * Errors: LL_ERR_INVALID_ARG for NULL or misaligned tensors (q, out and
+ * workspace 16-byte aligned, lse 4-byte aligned), first_frame < 0,
+ * n_query_frames < 1 or > n_local, softmax_scale negative or not finite, a q
+ * dtype that does not fit the cache, an invalid rope or cache descriptor, a
+ * workspace that is too small; LL_ERR_UNSUPPORTED for D other than 64 or
+ * 128 (BF16 and FP8 caches) or 64 (F32). All are reported before anything
+ * is launched.
  */
 size_t ll_sink_window_attention_workspace_bytes(const ll_kvcache* cache, int n_query_frames);
 
