@@ -234,3 +234,24 @@ def test_binding_rejects_host_tensors_and_mismatched_buffers(L):
         swa.kv_recache(cache, x, w, w, torch.ones(dout), 1e-6, [0, 1], rope)                  # 2 slots need 2N rows
     with pytest.raises(ValueError, match="whole number"):
         swa.rope_apply(torch.zeros(B, N + 1, H, D, dtype=torch.bfloat16), 0, rope)
+
+
+def test_workspace_sizes_and_noalloc_limit(L):
+    """Workspace = one arrival counter per unit (128 query rows of one head and
+    batch entry), then (#SMs + units) partial slots of 128 x D + 2 x 128 floats
+    (148 SMs: the count on a B200, and the fallback without a device); an FP8
+    cache adds the bf16 staging copy of K and V. The Wan frame (20 MB) and the
+    3-frame chunk (39 MB) fit the 48 MiB no-alloc scratch array."""
+    def ws(cache, nq):
+        return int(L.ll_sink_window_attention_workspace_bytes(ctypes.byref(cache), nq))
+    align = lambda x: (x + 255) // 256 * 256
+    slot = (128 * 128 + 2 * 128) * 4
+    for nq, units in [(1, 13 * 12), (3, 37 * 12)]:
+        want = align(align(units * 4) + (148 + units) * slot)
+        assert ws(_cache(), nq) == want
+        assert want <= 48 * 1024 * 1024
+    assert round(ws(_cache(), 1) / 1e6) == 20 and round(ws(_cache(), 3) / 1e6) == 39
+    fp8 = _cache(dtype=swa.LL_FP8_E4M3, k_scale=1 << 22, v_scale=1 << 23)
+    staging = 2 * align(12 * 1560 * 12 * 128 * 2)
+    assert ws(fp8, 1) == ws(_cache(), 1) + staging
+    assert ws(_cache(), 0) == 0 and L.ll_sink_window_attention_workspace_bytes(None, 1) == 0
