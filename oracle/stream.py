@@ -20,7 +20,7 @@ from typing import Dict, Optional, Sequence
 
 import numpy as np
 
-from .attention import mha
+from .attention import sink_window_attention
 from .recache import recache_frame
 from .rope import rope_3d, token_positions
 from .window import attended_frames
@@ -89,10 +89,7 @@ class StreamOracle:
         qr = self.rotate_queries(q, first_frame)
         if rows is not None:
             qr = qr[np.asarray(rows)]
-        frames = attended_frames(last, self.n_sink, self.n_local)
-        kk = np.concatenate([self.k[g] for g in frames], axis=0)
-        vv = np.concatenate([self.v[g] for g in frames], axis=0)
-        return mha(qr, kk, vv, scale, return_lse)
+        return sink_window_attention(qr, self.k, self.v, last, self.n_sink, self.n_local, scale, return_lse)
 
     def recache(self, switch_frame: int, x_by_frame: Dict[int, np.ndarray], wk, wv, gamma,
                 eps: float) -> None:

@@ -60,7 +60,6 @@ struct AttnTraits {
   static constexpr int MMA_K = 32 / ES;             // reduction elements per MMA
   static constexpr int FMT = (ES == 2) ? 1 : 2;     // bf16 / tf32
   static constexpr int QST = 2;                     // Q buffers
-  static constexpr int EXP_FMA_FROM = 8;            // pairs e with (e % 8) >= this use exp2_fma_x2 (8: none)
   static constexpr int CTRL_BYTES = 2048;
   static constexpr int STAGE_BUDGET = 232448 - CTRL_BYTES - 1024 - QST * Q_BYTES;
   static constexpr int STAGES = STAGE_BUDGET / KV_BYTES;
@@ -625,8 +624,8 @@ __global__ void __launch_bounds__(384, 1)
         }
         m_run = m_use;
         // p = 2^(s * scale * log2(e) - m) on pairs: the argument with one packed
-        // FMA, the exponential on the MUFU unit (optionally some pairs on the FMA
-        // pipe), the running sum in 4 packed partial sums
+        // FMA, the exponential on the MUFU unit, the running sum in 4 packed
+        // partial sums
         const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_use, -m_use);
         uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
@@ -635,15 +634,9 @@ __global__ void __launch_bounds__(384, 1)
           for (int e = 0; e < 16; ++e) {
             const uint64_t x2 =
                 f2_fma(f2_pack(__uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1])), sl2x2, negm2);
-            float a, a2;
-            if (TR::EXP_FMA_FROM < 8 && (e & 7) >= TR::EXP_FMA_FROM) {
-              exp2_fma_x2(x2, a, a2);
-            } else {
-              float x0, x1;
-              f2_unpack(x2, x0, x1);
-              a = ex2(x0);
-              a2 = ex2(x1);
-            }
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            const float a = ex2(x0), a2 = ex2(x1);
             ls2[e & 3] = f2_add(ls2[e & 3], f2_pack(a, a2));
             if constexpr (TR::ES == 2) {
               sr[c][e] = pack_bf16(a, a2);  // packed in place: slot e is free once 2e, 2e+1 were read

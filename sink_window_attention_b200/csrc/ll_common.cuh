@@ -488,33 +488,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
-// 2^x for two values on the FMA pipe instead of the MUFU unit.
-// Range reduction x = n + f with n = rint(x), taken with the 1.5 * 2^23
-// rounding constant (the sum's ulp is 1), and f in [-1/2, 1/2]; 2^f by a
-// cubic whose coefficients were fitted for minimal relative error on
-// [-1/2, 1/2] with Lawson's iteratively reweighted least squares (max
-// relative error 7.5e-5 with fp32 Horner evaluation, below the 2^-9 of the
-// bf16 P it feeds); n is then added to the exponent field. x is clamped at
-// -125 so every result is a normal number (2^-125 stands in for smaller
-// values, including -inf).
-__device__ __forceinline__ void exp2_fma_x2(uint64_t x, float& r0, float& r1) {
-  float x0, x1;
-  f2_unpack(x, x0, x1);
-  const uint64_t xc = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-  const uint64_t t = f2_add(xc, f2_pack(12582912.0f, 12582912.0f));
-  const uint64_t j = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
-  const uint64_t f = f2_fma(j, f2_pack(-1.0f, -1.0f), xc);
-  uint64_t p = f2_fma(f2_pack(0.0551716685295105f, 0.0551716685295105f), f,
-                      f2_pack(0.2426111400127411f, 0.2426111400127411f));
-  p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
-  p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
-  float p0, p1, t0, t1;
-  f2_unpack(p, p0, p1);
-  f2_unpack(t, t0, t1);
-  r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -87,6 +87,11 @@ def test_stream_matches_dense_masked_brute_force(n_local, chunk):
         ref = _dense_masked(Qr[f0 * N:(f0 + chunk) * N], Kr, V, np.repeat(np.arange(f0, f0 + chunk), N),
                             kframe, lambda qf, kf: kf in A, scale)
         assert np.allclose(got, ref, rtol=1e-11, atol=1e-11)
+        # the window function itself, fed per-frame rotated keys and values
+        kd = {g: Kr[g * N:(g + 1) * N] for g in range(last + 1)}
+        vd = {g: V[g * N:(g + 1) * N] for g in range(last + 1)}
+        direct = attention.sink_window_attention(Qr[f0 * N:(f0 + chunk) * N], kd, vd, last, 3, n_local)
+        assert np.allclose(direct, ref, rtol=1e-11, atol=1e-11)
         if n_local >= F:
             full = attention.frame_causal_attention(Qr, Kr, V, last, N)
             if chunk == 1:

@@ -282,6 +282,24 @@ def test_stream_pin_rejects_keys_rotated_at_their_slot(monkeypatch):
     assert rejected(pin)
 
 
+def window_attention_without_sinks(q_rot, k_rot_by_frame, v_by_frame, last_query_frame, n_sink=3, n_local=9,
+                                   scale=None, return_lse=False):
+    frames = [g for g in range(max(0, last_query_frame - n_local - n_sink + 1), last_query_frame + 1)]
+    k = np.concatenate([k_rot_by_frame[g] for g in frames], axis=0)
+    v = np.concatenate([v_by_frame[g] for g in frames], axis=0)
+    return attention.mha(q_rot, k, v, scale, return_lse)
+
+
+def test_window_attention_pin_rejects_missing_sinks(monkeypatch):
+    """The frame-set attention function (sink + window) is pinned against the
+    dense masked brute force: a version that attends to the last 12 frames
+    without the sinks is rejected."""
+    pin = [lambda: pin_att.test_stream_matches_dense_masked_brute_force(9, 1)]
+    assert not rejected(pin)
+    monkeypatch.setattr(attention, "sink_window_attention", window_attention_without_sinks)
+    assert rejected(pin)
+
+
 # ------------------------------------------------------------------ window and slots
 def attended_local_one_short(f, n_sink=3, n_local=9):
     if f < 0:
