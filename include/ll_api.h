@@ -270,8 +270,13 @@ ll_status ll_selftest_bounded_waits(void* stream);
  * the workspace and uses instead a scratch array of
  * LL_NOALLOC_SCRATCH_BYTES bytes that the library holds in static device
  * memory: every GPU that loads the library keeps it until the process exits.
+ * - `stream` must belong to the current device (LL_ERR_INVALID_ARG
+ *   otherwise): the array used is the current device's copy.
  * - The first call on a device looks up that device's copy of the array (with
- *   the device current); make that first call before any stream capture.
+ *   the device current); make that first call before any stream capture. The
+ *   address is kept for the life of the process: a cudaDeviceReset() (or any
+ *   teardown of the device's primary context) invalidates it, so do not call
+ *   this entry point again after one.
  * - Requests whose scratch need, ll_sink_window_attention_workspace_bytes(),
  *   exceeds LL_NOALLOC_SCRATCH_BYTES are rejected with LL_ERR_INVALID_ARG
  *   before anything is launched.

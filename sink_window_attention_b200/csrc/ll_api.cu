@@ -607,11 +607,16 @@ constexpr int kMaxDevices = kDeviceSlots;
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[kMaxDevices] = {};
 
-// Device address of the current device's scratch array (looked up once per
-// device, with that device current).
-ll_status noalloc_scratch(void** ptr) {
-  int dev = -1;
+// Device address of the scratch array of the device that `stream` belongs to,
+// which must be the current device (the address is looked up once per device,
+// with that device current).
+ll_status noalloc_scratch(cudaStream_t stream, void** ptr) {
+  int dev = -1, sdev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return check_launch("cudaGetDevice");
+  if (cudaStreamGetDevice(stream, &sdev) != cudaSuccess) return check_launch("cudaStreamGetDevice");
+  if (sdev != dev)
+    return fail(LL_ERR_INVALID_ARG, "the stream belongs to device %d but device %d is current; make the stream's "
+                                    "device current first", sdev, dev);
   if (dev < 0 || dev >= kMaxDevices) return fail(LL_ERR_UNSUPPORTED, "device ordinal %d is out of range", dev);
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
   if (g_noalloc_ptr[dev] == nullptr) {
@@ -640,7 +645,7 @@ ll_status ll_sink_window_attention_noalloc(const void* q, ll_dtype q_dtype, cons
                 "(use ll_sink_window_attention with a caller workspace)",
                 need, LL_NOALLOC_SCRATCH_BYTES);
   void* scratch = nullptr;
-  const ll_status st = noalloc_scratch(&scratch);
+  const ll_status st = noalloc_scratch(static_cast<cudaStream_t>(stream), &scratch);
   if (st != LL_OK) return st;
   return ll_sink_window_attention(q, q_dtype, cache, first_frame, n_query_frames, rope, softmax_scale, out, lse,
                                   scratch, LL_NOALLOC_SCRATCH_BYTES, stream);

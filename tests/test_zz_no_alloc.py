@@ -63,3 +63,26 @@ def test_noalloc_rejects_requests_beyond_the_static_scratch():
                                                     1 << 21, None, None)
     assert st == swa.LL_ERR_INVALID_ARG
     assert "static scratch" in swa.last_error()
+
+
+def test_noalloc_warm_call_allocates_no_device_memory():
+    """The point of the entry point: once the first call on the device has
+    looked up the static array, further calls take no device memory at all
+    (free memory as reported by cudaMemGetInfo is unchanged across them)."""
+    w = W.WAN
+    rope = swa.Rope(pairs=w.pairs, grid_h=w.grid_h, grid_w=w.grid_w, theta0=w.theta0)
+    cache = swa.KVCache(1, w.H, w.D, w.N, "bf16")
+    for f in range(12):
+        _, k, v = W.qkv_frames(w, 6, f, 1, device="cuda")
+        swa.kvcache_append(cache, k, v, f, rope)
+    q = W.qkv_frames(w, 6, 11, 1, device="cuda")[0]
+    out = torch.empty_like(q)
+    lse = torch.empty(1, w.H, w.N, device="cuda")
+    swa.sink_window_attention_noalloc(q, cache, 11, rope, out=out, lse=lse)   # first call: symbol lookup
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        swa.sink_window_attention_noalloc(q, cache, 11, rope, out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert swa.device_error() == 0
