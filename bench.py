@@ -207,30 +207,37 @@ class Stream:
             held[self.swa.slot_of_frame(f, w.n_sink, w.n_local)] = f
         return [f for f in held if f >= 0]
 
-    def step(self, seg: int, attn_events=None, qkv=None, recache_events=None):
-        """One 40-frame segment; frames 40*(seg+1) .. 40*(seg+1)+39, opened by a
-        prompt switch (recache of every layer)."""
+    def switch(self, first: int, recache_events=None) -> int:
+        """Prompt switch before frame `first`: the KV recache of every layer
+        (the cached frames re-projected from their hidden states with the new
+        prompt's projections). Returns the number of launches."""
         swa = self.swa
-        launches = 0
-        first = SEGMENT * (seg + 1)
         held = self.held_frames(first - 1)
         if recache_events is not None:
             recache_events[0].record()
         for l in range(self.layers):
             swa.kv_recache(self.caches[l], self.rx[l], self.rwk[l], self.rwv[l], self.rg[l], 1e-6, held, self.rope)
-            launches += 1
         if recache_events is not None:
             recache_events[1].record()
             recache_events[2].append((recache_events[0], recache_events[1]))
             recache_events[0] = torch.cuda.Event(enable_timing=True)
             recache_events[1] = torch.cuda.Event(enable_timing=True)
-        for i in range(SEGMENT):
-            f = SEGMENT * (seg + 1) + i
+        return self.layers
+
+    def frames(self, first: int, last: int, attn_events=None, qkv=None, on_output=None) -> int:
+        """Frames first .. last-1 through every layer: per frame and layer,
+        RoPE + append of the frame's K/V and attention of its queries (one
+        fused launch for a bf16 cache; append, then attention for an FP8
+        cache). on_output(f, layer, out) sees each attention output before
+        the next launch overwrites it. Returns the number of launches."""
+        swa = self.swa
+        launches = 0
+        for f in range(first, last):
             for l in range(self.layers):
                 if qkv is None:
                     q, k, v = self.q[l][f % POOL], self.k[l][f % POOL], self.v[l][f % POOL]
                 else:
-                    q, k, v = qkv(i, l)
+                    q, k, v = qkv(f, l)
                 fused = self.fused and self.caches[l].dtype != "fp8"
                 if not fused:
                     swa.kvcache_append(self.caches[l], k, v, f, self.rope)
@@ -241,15 +248,27 @@ class Stream:
                     swa.append_and_attend(self.caches[l], k, v, q, f, self.rope, out=self.out)
                 else:
                     swa.sink_window_attention(q, self.caches[l], f, self.rope, out=self.out)
-                if self.caches[l].dtype == "fp8":
-                    launches += 1  # the E4M3 -> bf16 staging kernel
+                launches += self.attention_launches(l)
                 if attn_events is not None:
                     attn_events[1].record()
                     attn_events[2].append((attn_events[0], attn_events[1]))
                     attn_events[0] = torch.cuda.Event(enable_timing=True)
                     attn_events[1] = torch.cuda.Event(enable_timing=True)
-                launches += 1
+                if on_output is not None:
+                    on_output(f, l, self.out)
         return launches
+
+    def attention_launches(self, layer: int) -> int:
+        """Kernel launches of one attention call on this layer's cache (an
+        E4M3 cache: the staging dequantisation, then the attention kernel)."""
+        return 2 if self.caches[layer].dtype == "fp8" else 1
+
+    def step(self, seg: int, attn_events=None, recache_events=None) -> int:
+        """One 40-frame segment: frames 40*(seg+1) .. 40*(seg+1)+39, opened by
+        a prompt switch (recache of every layer)."""
+        first = SEGMENT * (seg + 1)
+        launches = self.switch(first, recache_events)
+        return launches + self.frames(first, first + SEGMENT, attn_events)
 
 
 def run_ours(args, rank, world, local_rank):
@@ -310,7 +329,8 @@ def run_ours(args, rank, world, local_rank):
     fl = attention_flops(w)
     achieved = fl / avg_attn_s / 1e12
     # the timed launch is the fused append + attention in the default stream
-    traffic = load_traffic("attention_fused_stream.md" if fused else "attention_wan_single_layer.md")
+    traffic_capture = "attention_fused_stream" if fused else "attention_wan_single_layer"
+    traffic = load_traffic(traffic_capture)
     recache_ms = [a.elapsed_time(b) for a, b in rev[2]]
     rc_layer_s = (sum(recache_ms) / len(recache_ms)) / 1e3 / w.layers
     rc_flops = 2.0 * (w.slots * w.N) * w.dm * (2 * w.H * w.D)
@@ -330,6 +350,9 @@ def run_ours(args, rank, world, local_rank):
                          " (the frame's RoPE + append fused in: ll_append_and_attend)" if fused else ""),
                      "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "traffic_source": (f"ncu capture '{traffic_capture}' of this kernel version "
+                                        "(profiles/traffic.json), not measured in this run"
+                                        if traffic is not None else "no capture of this kernel version"),
                      "peak_kind": f"{kind} bf16 dense, sustained",
                      "algorithmic_flops_per_launch": fl, "avg_launch_us": round(avg_attn_s * 1e6, 2)},
         "recache_kernel": {"achieved_tflops": round(rc_flops / rc_layer_s / 1e12, 1),
@@ -339,7 +362,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = cpu_baseline(w)
     return line
 
 
@@ -430,20 +453,19 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def load_traffic(profile: str = "attention_wan_single_layer.md"):
-    """DRAM bytes (read + write) per attention launch from a committed ncu
-    summary — only while the kernel sources still hash to the captured
-    version; otherwise null."""
-    p = os.path.join(ROOT, "profiles", profile)
+def load_traffic(capture: str):
+    """DRAM bytes (read + write) per launch of one ncu capture, from the
+    committed data file profiles/traffic.json — a figure taken by ncu on an
+    earlier run, not a measurement of this run — and only while the kernel
+    sources still hash to the version that capture names; otherwise None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
-    text = open(p).read()
-    import re
-    m_hash = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
-    m_bytes = re.search(r"dram_bytes_per_launch[^|]*\|\s*([0-9]+)", text)
-    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+    with open(p) as f:
+        rec = json.load(f).get(capture)
+    if not rec or rec.get("kernel_source_sha256_16") != kernel_source_hash():
         return None
-    return int(m_bytes.group(1))
+    return int(rec["dram_bytes_per_launch"])
 
 
 # ---------------------------------------------------------------------------
@@ -473,17 +495,15 @@ class OracleStep:
                        self.rng.standard_normal((w.N, w.H, w.D)) * w.qkv_scale)
         self.f += 1
 
-    def time(self, rows: int):
-        """(seconds for the sample, seconds extrapolated to the full layer-step)."""
+    def time(self, rows: int) -> float:
+        """Seconds for one sample: the append of one frame and the attention
+        of its first `rows` query rows."""
         w = self.w
         q = self.rng.standard_normal((w.N, w.H, w.D)) * w.qkv_scale
         t0 = time.perf_counter()
         self._append()
-        t_append = time.perf_counter() - t0
-        t0 = time.perf_counter()
         self.so.attend(q, self.f - 1, rows=np.arange(rows))
-        t_attn = time.perf_counter() - t0
-        return t_append + t_attn, t_append + t_attn * (w.N / rows)
+        return time.perf_counter() - t0
 
 
 def blas_threads() -> int:
@@ -497,44 +517,72 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
-def cpu_baseline(w: W.Workload, budget_s: float = 20.0):
+# The oracle's sample, shared by the cpu_baseline of our arm and every step of
+# the reference arm: one steady-state layer-step (append of one latent frame
+# and attention of its query rows over the 12-frame window), restricted to the
+# first `rows` query rows so that one sample takes about STEP_TARGET_S on the
+# host (all rows when the host is fast enough). One whole layer-step is one of
+# the 30 layers of one latent frame; the per-segment recache (1/40 of a
+# layer's recache per layer-step, under 1 % of the work) is not included.
+STEP_TARGET_S = 3.0
+
+
+def oracle_rows(ora: "OracleStep") -> int:
+    """Query rows per sample: a 64-row probe (the faster of two, the first
+    pays for page faults) scaled to STEP_TARGET_S."""
+    t64 = min(ora.time(64), ora.time(64))
+    return int(max(64, min(ora.w.N, 64 * STEP_TARGET_S / max(t64, 1e-3))))
+
+
+def oracle_sample_desc(w: W.Workload, rows: int) -> str:
+    return (f"one steady-state layer-step in float64 NumPy restricted to {rows} of its {w.N} query rows: append "
+            f"of 1 latent frame and attention of those rows, all {w.H} heads, over {w.slots * w.N} keys; "
+            f"= {rows}/{w.N} x 1/{w.layers} of one latent frame through the {w.layers}-layer stack (the recache, "
+            f"under 1 % of the work, not included)")
+
+
+def oracle_frames(w: W.Workload, rows: int) -> float:
+    """Latent frames of stack work that one sample of `rows` rows amounts to."""
+    return rows / w.N / w.layers
+
+
+def cpu_baseline(w: W.Workload):
     ora = OracleStep(w)
-    rows = 64
-    sample_s, full_s = ora.time(rows)
-    if sample_s < budget_s / 4:      # grow the sample towards the budget
-        rows = int(min(w.N, rows * max(1.0, (budget_s / 2) / max(sample_s, 1e-3))))
-        sample_s, full_s = ora.time(rows)
-    frames_per_s = 1.0 / (full_s * w.layers)
-    return {"value": round(frames_per_s, 6), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"one steady-state layer-step (append of 1 frame + attention of {rows} of 1560 query rows, "
-                      f"all 12 heads, 18720 keys) in float64 NumPy; took {sample_s:.2f} s; extrapolated to the "
-                      f"full layer-step ({full_s:.2f} s) and to {w.layers} layers"}
+    rows = oracle_rows(ora)
+    t = ora.time(rows)
+    return {"value": round(oracle_frames(w, rows) / t, 6), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{oracle_sample_desc(w, rows)}; took {t:.2f} s"}
 
 
 def run_reference(args, rank, world):
+    """The oracle on the host cores, timed as it runs: every step is one
+    oracle sample and ms_per_step is its measured wall time; value is the
+    latent frames that work amounts to per second."""
     if rank != 0:
         return None
     w = W.STREAM
-    rows = 128
     ora = OracleStep(w)
+    rows = oracle_rows(ora)
     samples = []
     for s in range(args.warmup + args.steps):
-        _, full_s = ora.time(rows)
+        t = ora.time(rows)
         if s >= args.warmup:
-            samples.append(full_s)
-    per_frame = statistics.mean(samples) * w.layers
-    value = 1.0 / per_frame
-    sample = (f"each step: the oracle (float64 NumPy) on one steady-state layer-step, {rows} of 1560 query rows, "
-              f"extrapolated to the full layer-step and {w.layers} layers")
-    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_frame * 1e3, 3),
+            samples.append(t)
+    step_s = statistics.mean(samples)
+    value = oracle_frames(w, rows) / step_s
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 7), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"240s stream segment: latent frames x {w.layers} layers, H=12 D=128, "
                                    "1560 tok/frame, 3 sink + 9 local, LoL jitter 0.8",
+                       "step": f"{rows}/{w.N} of one layer-step = {oracle_frames(w, rows):.3g} latent frame",
                        "parallelism": "host cores"},
-            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                             "sample": sample},
-            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "extrapolated": {"ms_per_latent_frame": round(step_s / oracle_frames(w, rows) * 1e3, 1),
+                             "note": "the measured step time scaled to a whole latent frame through the stack "
+                                     "(rows and layers); not a measurement"},
+            "cpu_baseline": {"value": round(value, 7), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": oracle_sample_desc(w, rows)},
+            "e2e": {"value": round(value, 7), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
 def run_attention_only(args):
@@ -577,14 +625,18 @@ def run_attention_only(args):
 
 
 def run_append_only(args):
-    """One Wan frame's RoPE + append into a layer cache (bf16 or E4M3 cache):
-    `warmup` + `steps` launches, each after a 256 MB write that evicts L2,
-    timed with CUDA events; achieved HBM bandwidth from the algorithmic bytes."""
+    """RoPE + append of one Wan frame (or a 3-frame chunk with --workload
+    chunk) into a layer cache (bf16 or E4M3 cache): `warmup` + `steps`
+    launches, each after a 256 MB write that evicts L2, timed with CUDA
+    events; achieved HBM bandwidth from the algorithmic bytes."""
     from sink_window_attention_b200 import build
     build.build()
     import sink_window_attention_b200 as swa
-    w = W.WAN
+    w = W.WAN if args.workload == "wan" else W.CHUNK
+    c = w.query_frames
     st = Stream(W.replace(w, layers=1, sigma_t=0.8, jitter_seed=4), args.cache, "cuda")
+    ks = [W.normal((1, c * w.N, w.H, w.D), 50 + i, w.qkv_scale, torch.bfloat16, "cuda") for i in range(2)]
+    vs = [W.normal((1, c * w.N, w.H, w.D), 60 + i, w.qkv_scale, torch.bfloat16, "cuda") for i in range(2)]
     flush = torch.empty(64 << 20, dtype=torch.float32, device="cuda")
     f0 = 3 * 40
     ev = []
@@ -593,16 +645,56 @@ def run_append_only(args):
         flush.zero_()
         torch.cuda._sleep(200_000)
         a.record()
-        swa.kvcache_append(st.caches[0], st.k[0][i % POOL], st.v[0][i % POOL], f0 + i, st.rope)
+        swa.kvcache_append(st.caches[0], ks[i % 2], vs[i % 2], f0 + c * i, st.rope)
         b.record()
         ev.append((a, b))
     torch.cuda.synchronize()
     times = [a.elapsed_time(b) / 1e3 for a, b in ev[args.warmup:]]
     assert swa.device_error() == 0
-    nbytes = append_bytes(w, 1 if args.cache == "fp8" else 2)
+    nbytes = c * append_bytes(w, 1 if args.cache == "fp8" else 2)
     peaks, kind = measured_peaks()
     t = statistics.median(times)
-    return {"mode": "append", "cache": args.cache, "launches": len(times), "median_us": round(t * 1e6, 2),
+    return {"mode": "append", "workload": w.name, "frames": c, "cache": args.cache, "launches": len(times),
+            "median_us": round(t * 1e6, 2), "algorithmic_bytes": nbytes, "gbs": round(nbytes / t / 1e9, 1),
+            "frac_of_hbm_peak": round(nbytes / t / 1e9 / peaks["hbm_gbs"], 4), "peak_kind": kind}
+
+
+def rope_bytes(w: W.Workload, frames: int) -> float:
+    """Algorithmic HBM bytes of an in-place RoPE of `frames` frames of one
+    bf16 [N, H, D] tensor: every element read once and written once."""
+    return 2.0 * 2 * frames * w.N * w.H * w.D
+
+
+def run_rope_only(args):
+    """In-place RoPE (ll_rope_apply) of one Wan frame's Q (or a 3-frame chunk
+    with --workload chunk): `warmup` + `steps` launches, each after a 256 MB
+    write that evicts L2, timed with CUDA events; achieved HBM bandwidth from
+    the algorithmic bytes."""
+    from sink_window_attention_b200 import build
+    build.build()
+    import sink_window_attention_b200 as swa
+    w = W.replace(W.WAN if args.workload == "wan" else W.CHUNK, sigma_t=0.8, jitter_seed=4)
+    c = w.query_frames
+    rope = swa.Rope(pairs=w.pairs, grid_h=w.grid_h, grid_w=w.grid_w, theta0=w.theta0, sigma_t=w.sigma_t,
+                    eps=[float(e) for e in w.eps], t_offset=w.t_offset)
+    xs = [W.normal((1, c * w.N, w.H, w.D), 70 + i, w.qkv_scale, torch.bfloat16, "cuda") for i in range(2)]
+    flush = torch.empty(64 << 20, dtype=torch.float32, device="cuda")
+    ev = []
+    for i in range(args.warmup + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        flush.zero_()
+        torch.cuda._sleep(200_000)
+        a.record()
+        swa.rope_apply(xs[i % 2], 120 + c * i, rope)
+        b.record()
+        ev.append((a, b))
+    torch.cuda.synchronize()
+    times = [a.elapsed_time(b) / 1e3 for a, b in ev[args.warmup:]]
+    assert swa.device_error() == 0
+    nbytes = rope_bytes(w, c)
+    peaks, kind = measured_peaks()
+    t = statistics.median(times)
+    return {"mode": "rope", "workload": w.name, "frames": c, "launches": len(times), "median_us": round(t * 1e6, 2),
             "algorithmic_bytes": nbytes, "gbs": round(nbytes / t / 1e9, 1),
             "frac_of_hbm_peak": round(nbytes / t / 1e9 / peaks["hbm_gbs"], 4), "peak_kind": kind}
 
@@ -644,8 +736,7 @@ def main():
     ap.add_argument("--layers", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--separate", action="store_true", help="append and attention as two calls (bf16 cache)")
-    ap.add_argument("--cpu-budget", type=float, default=20.0)
-    ap.add_argument("--mode", default="stream", choices=["stream", "attention", "recache", "append"])
+    ap.add_argument("--mode", default="stream", choices=["stream", "attention", "recache", "append", "rope"])
     ap.add_argument("--workload", default="wan", choices=["wan", "chunk"])
     args = ap.parse_args()
     if args.mode == "attention":
@@ -656,6 +747,9 @@ def main():
         return
     if args.mode == "append":
         print(json.dumps(run_append_only(args)), flush=True)
+        return
+    if args.mode == "rope":
+        print(json.dumps(run_rope_only(args)), flush=True)
         return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -53,16 +53,18 @@ def test_recache_recomputes_exactly_the_cached_frames():
 
 
 def test_traffic_figure_only_for_the_captured_kernel(tmp_path, monkeypatch):
-    """The bench line's roofline.traffic comes from a committed ncu summary only
-    while the attention sources hash to the version that summary names;
-    otherwise it is null (a stale DRAM figure is never reported)."""
+    """The bench line's roofline.traffic comes from the committed capture file
+    profiles/traffic.json only while the attention sources hash to the version
+    that capture names; otherwise it is null (a stale DRAM figure is never
+    reported)."""
+    import json
     prof = tmp_path / "profiles"
     prof.mkdir()
-    (prof / "k.md").write_text("kernel_source_sha256_16: 0123456789abcdef\n\n"
-                               "| dram_bytes_per_launch (read + write) | 230756864 |\n")
+    (prof / "traffic.json").write_text(json.dumps(
+        {"k": {"kernel_source_sha256_16": "0123456789abcdef", "dram_bytes_per_launch": 230756864}}))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0123456789abcdef")
-    assert bench.load_traffic("k.md") == 230756864
+    assert bench.load_traffic("k") == 230756864
+    assert bench.load_traffic("missing") is None
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "fedcba9876543210")
-    assert bench.load_traffic("k.md") is None
-    assert bench.load_traffic("missing.md") is None
+    assert bench.load_traffic("k") is None
