@@ -238,7 +238,7 @@ class Stream:
                     q, k, v = self.q[l][f % POOL], self.k[l][f % POOL], self.v[l][f % POOL]
                 else:
                     q, k, v = qkv(f, l)
-                fused = self.fused and self.caches[l].dtype != "fp8"
+                fused = self.fuses(l)
                 if not fused:
                     swa.kvcache_append(self.caches[l], k, v, f, self.rope)
                     launches += 1
@@ -257,6 +257,11 @@ class Stream:
                 if on_output is not None:
                     on_output(f, l, self.out)
         return launches
+
+    def fuses(self, layer: int) -> bool:
+        """Whether this layer's frames run as one fused append + attention
+        launch (bf16 and f32 caches; an E4M3 cache takes the two calls)."""
+        return self.fused and self.caches[layer].dtype != "fp8"
 
     def attention_launches(self, layer: int) -> int:
         """Kernel launches of one attention call on this layer's cache (an
@@ -280,7 +285,7 @@ def run_ours(args, rank, world, local_rank):
     w = W.replace(w, layers=args.layers)
     st = Stream(w, "bf16" if args.cache == "bf16" else "fp8", "cuda", seed_offset=replica_seed_offset(rank),
                 fused=not args.separate)
-    fused = st.fused and args.cache == "bf16"
+    fused = st.fuses(0)
     dist = world > 1
     if dist:
         import torch.distributed as tdist
@@ -329,7 +334,8 @@ def run_ours(args, rank, world, local_rank):
     fl = attention_flops(w)
     achieved = fl / avg_attn_s / 1e12
     # the timed launch is the fused append + attention in the default stream
-    traffic_capture = "attention_fused_stream" if fused else "attention_wan_single_layer"
+    traffic_capture = ("attention_fused_stream" if fused else "attention_wan_single_layer") + (
+        "_fp8" if args.cache == "fp8" else "")
     traffic = load_traffic(traffic_capture)
     recache_ms = [a.elapsed_time(b) for a, b in rev[2]]
     rc_layer_s = (sum(recache_ms) / len(recache_ms)) / 1e3 / w.layers
@@ -346,8 +352,8 @@ def run_ours(args, rank, world, local_rank):
                    "recache": f"all {w.layers} layers at the segment start (X [{w.slots * w.N}, {w.dm}])",
                    "l2": "inputs larger than L2 (30 caches x 115 MB)", "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "tensor", "kernel": "sink_window_attention_kernel" + (
-                         " (+ E4M3 staging kernel inside the timed call)" if args.cache == "fp8" else
-                         " (the frame's RoPE + append fused in: ll_append_and_attend)" if fused else ""),
+                         " (the frame's RoPE + append fused in: ll_append_and_attend)" if fused else "") + (
+                         " (+ the E4M3 -> bf16 staging kernel inside the timed call)" if args.cache == "fp8" else ""),
                      "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "traffic_source": (f"ncu capture '{traffic_capture}' of this kernel version "
@@ -358,6 +364,7 @@ def run_ours(args, rank, world, local_rank):
         "recache_kernel": {"achieved_tflops": round(rc_flops / rc_layer_s / 1e12, 1),
                            "us_per_layer": round(rc_layer_s * 1e6, 2), "flops_per_layer": rc_flops},
         "e2e": e2e,
+        "hbm_kernels": hbm_kernels(args.cache),
         "gpu_launches": launches,
         "clocks": clk,
     }
@@ -417,7 +424,7 @@ def run_e2e(st: Stream, args, barrier, dist):
             f = SEGMENT * (s + 1) + i
             for l in range(L):
                 q, k, v = dev[b][l]
-                if st.fused and st.caches[l].dtype != "fp8":
+                if st.fuses(l):
                     st.swa.append_and_attend(st.caches[l], k, v, q, f, st.rope, out=st.out)
                 else:
                     st.swa.kvcache_append(st.caches[l], k, v, f, st.rope)
@@ -657,6 +664,21 @@ def run_append_only(args):
     return {"mode": "append", "workload": w.name, "frames": c, "cache": args.cache, "launches": len(times),
             "median_us": round(t * 1e6, 2), "algorithmic_bytes": nbytes, "gbs": round(nbytes / t / 1e9, 1),
             "frac_of_hbm_peak": round(nbytes / t / 1e9 / peaks["hbm_gbs"], 4), "peak_kind": kind}
+
+
+def hbm_kernels(cache: str):
+    """The HBM-bound kernels timed alone (each launch after an L2 flush): the
+    RoPE + append of one Wan frame and of a 3-frame chunk into this run's
+    cache type, and the in-place RoPE of the same Q sizes. In the stream the
+    append is fused into the attention launch and the Q rotation into its Q
+    load, so these are the separate entry points' figures."""
+    out = {}
+    for wl in ("wan", "chunk"):
+        a = argparse.Namespace(workload=wl, cache=cache, steps=10, warmup=3)
+        for name, fn in (("append", run_append_only), ("rope", run_rope_only)):
+            r = fn(a)
+            out[f"{name}_{wl}"] = {k: r[k] for k in ("median_us", "algorithmic_bytes", "gbs", "frac_of_hbm_peak")}
+    return out
 
 
 def rope_bytes(w: W.Workload, frames: int) -> float:

@@ -33,6 +33,7 @@ def test_noalloc_matches_workspace_entry_point():
     rope = swa.Rope(pairs=w.pairs, grid_h=w.grid_h, grid_w=w.grid_w, theta0=w.theta0, sigma_t=0.8,
                     eps=[float(e) for e in eps])
     cache = swa.KVCache(1, w.H, w.D, w.N, "bf16")
+    assert swa.attention_workspace_bytes(cache, 1) <= swa.NOALLOC_SCRATCH_BYTES
     for f in range(12):
         _, k, v = W.qkv_frames(w, 5, f, 1, device="cuda")
         swa.kvcache_append(cache, k, v, f, rope)
@@ -49,6 +50,19 @@ def test_noalloc_matches_workspace_entry_point():
             assert_parity(out.double().cpu().numpy(), ref.double().cpu().numpy(), what=f"noalloc frame {f}")
             assert_parity(lse.cpu().numpy(), lse_ref.cpu().numpy(), max_rel=1e-3, mean_abs=5e-3, what="lse")
     assert swa.device_error() == 0
+
+
+def test_noalloc_rejects_an_fp8_wan_cache():
+    """Attention over an E4M3 cache reads a bf16 staging copy of the occupied
+    rows (about 115 MB for the Wan-shaped layer) that lives in the scratch:
+    far beyond the static array, so the call is refused before any launch."""
+    w = W.WAN
+    cache = swa.KVCache(1, w.H, w.D, w.N, "fp8")
+    assert swa.attention_workspace_bytes(cache, 1) > swa.NOALLOC_SCRATCH_BYTES
+    q = torch.zeros(1, w.N, w.H, w.D, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(swa.LLError) as e:
+        swa.sink_window_attention_noalloc(q, cache, 20, None)
+    assert e.value.status == swa.LL_ERR_INVALID_ARG and "static scratch" in str(e.value)
 
 
 def test_noalloc_rejects_requests_beyond_the_static_scratch():
