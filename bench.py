@@ -360,7 +360,11 @@ def run_ours(args, rank, world, local_rank):
                                         "(profiles/traffic.json), not measured in this run"
                                         if traffic is not None else "no capture of this kernel version"),
                      "peak_kind": f"{kind} bf16 dense, sustained",
-                     "algorithmic_flops_per_launch": fl, "avg_launch_us": round(avg_attn_s * 1e6, 2)},
+                     "algorithmic_flops_per_launch": fl, "avg_launch_us": round(avg_attn_s * 1e6, 2),
+                     # the launch time in SM clock cycles at the run's median clock: separates a
+                     # slower clock (power cap) from more work per launch when runs are compared
+                     "avg_launch_kcycles_at_median_clock": (round(avg_attn_s * clk["sm_mhz"] * 1e3, 1)
+                                                            if clk and clk.get("sm_mhz") else None)},
         "recache_kernel": {"achieved_tflops": round(rc_flops / rc_layer_s / 1e12, 1),
                            "us_per_layer": round(rc_layer_s * 1e6, 2), "flops_per_layer": rc_flops},
         "e2e": e2e,
