@@ -210,16 +210,20 @@ ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvc
  * "Short-Window Attention": a new frame enters the window and attends to it).
  * The results equal those of the two calls made one after the other.
  * k, v, q, out: [B][n_frames*N][H][D] of `dtype`, which must be the cache's
- * dtype (BF16 or F32; an FP8 cache needs the two separate calls). The other
- * arguments are those of the two calls. workspace: device scratch of at least
+ * dtype (BF16 or F32), or BF16 for an FP8 cache. The other arguments are those
+ * of the two calls. workspace: device scratch of at least
  * ll_append_and_attend_workspace_bytes(...) bytes, its contents need not be
  * initialised (the grid barrier word is tagged with a per-launch generation,
  * so it never needs resetting), and calls sharing it must be ordered.
- * The launch is cooperative: every CTA must be resident at once, otherwise
- * the launch fails with LL_ERR_CUDA instead of running.
- * Errors: those of the two calls; LL_ERR_UNSUPPORTED for an FP8 cache or D
- * other than 64 / 128 (bf16) and 64 (f32); LL_ERR_TIMEOUT (from
- * ll_device_error) when the barrier wait gives up.
+ * BF16 / F32 cache: one cooperative launch; every CTA must be resident at
+ * once, otherwise the launch fails with LL_ERR_CUDA instead of running.
+ * FP8 cache: two launches; the first appends the new frames (codes and scales
+ * into their slots) and writes the bf16 staging copy of every occupied row
+ * that attention over an FP8 cache reads (the new frames' rows from the
+ * codes just written), the second is the bf16 attention over that copy.
+ * Errors: those of the two calls; LL_ERR_UNSUPPORTED for D other than 64 /
+ * 128 (bf16, FP8) and 64 (f32) and for an FP8 cache of more than 64 slots;
+ * LL_ERR_TIMEOUT (from ll_device_error) when the barrier wait gives up.
  */
 size_t ll_append_and_attend_workspace_bytes(const ll_kvcache* cache, int n_frames);
 

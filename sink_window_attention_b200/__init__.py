@@ -306,7 +306,8 @@ def append_and_attend(cache: KVCache, k: torch.Tensor, v: torch.Tensor, q: torch
                       lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
                       stream=None) -> torch.Tensor:
     """ll_append_and_attend: append frames first_frame.. (k, v [B, F*N, H, D])
-    and attend with their queries q in one kernel (BF16 / F32 caches)."""
+    and attend with their queries q (one kernel for BF16 / F32 caches; for an
+    E4M3 cache the append with the bf16 staging copy, then attention)."""
     F = _check_shape(cache, q, "q")
     if _check_shape(cache, k, "k") != F or _check_shape(cache, v, "v") != F:
         raise ValueError("k, v and q must cover the same frames")

@@ -275,6 +275,67 @@ size_t attention_scratch_bytes(const ll_kvcache* cache, int n_query_frames) {
   return align256(attention_workspace<ll::AttnTraits<64, __nv_bfloat16>>(units));
 }
 
+ll_status launch_bf16_attention_on(const ll_kvcache* staged, const void* q, long long first_frame, int n_query_frames,
+                                   const ll_rope_desc* rope, float softmax_scale, void* out, float* lse,
+                                   void* workspace, size_t workspace_bytes, cudaStream_t s);
+
+// The fused append + attention over an E4M3 cache: one kernel appends the new
+// frames (codes and scales into their slots, their dequantised values into
+// the bf16 staging rows) and dequantises every other occupied row into the
+// staging copy; the bf16 attention kernel then reads the staging copy. The
+// results equal those of ll_kvcache_append followed by
+// ll_sink_window_attention.
+ll_status append_stage_and_attend(const ll_kvcache* cache, const ll::AppendParams& ap, const void* q,
+                                  long long first_frame, int n_frames, const ll_rope_desc* rope, float softmax_scale,
+                                  void* out, float* lse, void* workspace, size_t workspace_bytes, cudaStream_t s) {
+  const long long S = cache->n_sink + cache->n_local;
+  const long long last = first_frame + n_frames - 1;
+  const long long valid_slots = last + 1 < S ? last + 1 : S;
+  const size_t half = fp8_staging_half(cache);
+  char* stage = static_cast<char*>(workspace) + attention_scratch_bytes(cache, n_frames);
+  ll::AppendStageParams q8{};
+  q8.ap = ap;
+  q8.ap.stage_k = reinterpret_cast<__nv_bfloat16*>(stage);
+  q8.ap.stage_v = reinterpret_cast<__nv_bfloat16*>(stage + half);
+  ll::DequantParams& dp = q8.dq;
+  dp.src[0] = static_cast<const uint8_t*>(cache->k);
+  dp.src[1] = static_cast<const uint8_t*>(cache->v);
+  dp.scale[0] = cache->k_scale;
+  dp.scale[1] = cache->v_scale;
+  dp.dst[0] = q8.ap.stage_k;
+  dp.dst[1] = q8.ap.stage_v;
+  dp.B = cache->B;
+  dp.rows = static_cast<int>(valid_slots * cache->tokens_per_frame);
+  dp.batch_rows = static_cast<int>(S * cache->tokens_per_frame);
+  dp.H = cache->H;
+  dp.D = cache->D;
+  for (int i = 0; i < n_frames; ++i) {
+    int slot = 0;
+    ll_slot_of_frame(first_frame + i, cache->n_sink, cache->n_local, &slot);
+    q8.new_slots |= 1ull << slot;
+  }
+  const long long threads = ll::append_items(ap);
+  const long long want_a = (threads + 255) / 256;
+  q8.append_blocks = static_cast<int>(want_a < 8LL * num_sms() ? want_a : 8LL * num_sms());
+  const long long chunks = static_cast<long long>(dp.B) * dp.rows * dp.H * (dp.D / 16);
+  const long long want_d = (chunks + 255) / 256;
+  q8.dequant_blocks = static_cast<int>(want_d < 4LL * num_sms() ? want_d : 4LL * num_sms());
+  const size_t smem = ll::append_smem_bytes(n_frames, cache->H, cache->D, ap.rp.pt);
+  if (smem > 48 * 1024)
+    return fail(LL_ERR_UNSUPPORTED, "frequency tables of %zu bytes exceed 48 KiB (n_frames x H x pairs_t too large)",
+                smem);
+  ll::append_stage_e4m3_kernel<<<q8.append_blocks + 2 * q8.dequant_blocks, 256, smem, s>>>(q8);
+  ll_status st = check_launch("append_stage_e4m3_kernel");
+  if (st != LL_OK) return st;
+  ll_kvcache staged = *cache;
+  staged.k = q8.ap.stage_k;
+  staged.v = q8.ap.stage_v;
+  staged.k_scale = staged.v_scale = nullptr;
+  staged.dtype = LL_BF16;
+  return launch_bf16_attention_on(&staged, q, first_frame, n_frames, rope, softmax_scale, out, lse, workspace,
+                                  workspace_bytes, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -474,11 +535,40 @@ ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvc
   return fail(LL_ERR_UNSUPPORTED, "attention supports D = 64 or 128 (bf16) and D = 64 (f32); got D = %d", cache->D);
 }
 
+}  // extern "C"
+
+namespace {
+// The bf16 attention kernel over a bf16 cache descriptor (validated by the caller).
+ll_status launch_bf16_attention_on(const ll_kvcache* staged, const void* q, long long first_frame, int n_query_frames,
+                                   const ll_rope_desc* rope, float softmax_scale, void* out, float* lse,
+                                   void* workspace, size_t workspace_bytes, cudaStream_t s) {
+  const long long S = staged->n_sink + staged->n_local;
+  const long long last = first_frame + n_query_frames - 1;
+  const long long valid_slots = last + 1 < S ? last + 1 : S;
+  ll::AttnParams p{};
+  ll_status st = make_rope(rope, staged->H, staged->D, first_frame, &p.rp);
+  if (st != LL_OK) return st;
+  p.q = q;
+  p.out = out;
+  p.lse = lse;
+  p.B = staged->B;
+  p.H = staged->H;
+  p.Tq = n_query_frames * staged->tokens_per_frame;
+  p.Nk = static_cast<int>(valid_slots * staged->tokens_per_frame);
+  p.softmax_scale = softmax_scale;
+  p.N = staged->tokens_per_frame;
+  if (staged->D == 128)
+    return launch_attention<ll::AttnTraits<128, __nv_bfloat16>>(p, staged, S, workspace, workspace_bytes, s);
+  return launch_attention<ll::AttnTraits<64, __nv_bfloat16>>(p, staged, S, workspace, workspace_bytes, s);
+}
+}  // namespace
+
+extern "C" {
+
 size_t ll_append_and_attend_workspace_bytes(const ll_kvcache* cache, int n_frames) {
-  if (cache == nullptr || n_frames < 1 || cache->tokens_per_frame < 1 || cache->H < 1 || cache->B < 1 ||
-      cache->dtype == LL_FP8_E4M3)
-    return 0;
-  return attention_scratch_bytes(cache, n_frames) + 256;  // + the grid barrier word
+  if (cache == nullptr || n_frames < 1 || cache->tokens_per_frame < 1 || cache->H < 1 || cache->B < 1) return 0;
+  // + the grid barrier word; an FP8 cache: + the bf16 staging copy instead
+  return attention_scratch_bytes(cache, n_frames) + (cache->dtype == LL_FP8_E4M3 ? fp8_staging_bytes(cache) : 256);
 }
 
 ll_status ll_append_and_attend(const ll_kvcache* cache, const void* k, const void* v, const void* q, ll_dtype dtype,
@@ -487,10 +577,13 @@ ll_status ll_append_and_attend(const ll_kvcache* cache, const void* k, const voi
   g_last_error.clear();
   ll_status st = check_cache(cache);
   if (st != LL_OK) return st;
-  if (cache->dtype == LL_FP8_E4M3)
-    return fail(LL_ERR_UNSUPPORTED, "the fused append + attention takes a BF16 or F32 cache (FP8: call "
-                                    "ll_kvcache_append, then ll_sink_window_attention)");
-  if (dtype != cache->dtype) return fail(LL_ERR_INVALID_ARG, "k, v and q must have the cache's dtype");
+  const bool fp8 = cache->dtype == LL_FP8_E4M3;
+  if (fp8 ? dtype != LL_BF16 : dtype != cache->dtype)
+    return fail(LL_ERR_INVALID_ARG, "k, v and q must have the cache's dtype (BF16 for an FP8 cache)");
+  if (fp8 && cache->D != 128 && cache->D != 64)
+    return fail(LL_ERR_UNSUPPORTED, "attention supports D = 64 or 128; got D = %d", cache->D);
+  if (fp8 && cache->n_sink + cache->n_local > 64)
+    return fail(LL_ERR_UNSUPPORTED, "the fused append over an FP8 cache takes at most 64 slots");
   if (k == nullptr || v == nullptr || q == nullptr || out == nullptr)
     return fail(LL_ERR_INVALID_ARG, "k, v, q and out must be non-NULL");
   if (!aligned16(k) || !aligned16(v) || !aligned16(q) || !aligned16(out))
@@ -517,6 +610,8 @@ ll_status ll_append_and_attend(const ll_kvcache* cache, const void* k, const voi
   ap.v_in = v;
   ap.k_cache = cache->k;
   ap.v_cache = cache->v;
+  ap.k_scale = cache->k_scale;
+  ap.v_scale = cache->v_scale;
   ap.B = cache->B;
   ap.F = n_frames;
   ap.N = cache->tokens_per_frame;
@@ -527,6 +622,8 @@ ll_status ll_append_and_attend(const ll_kvcache* cache, const void* k, const voi
   ap.first_frame = first_frame;
   if (ll::append_items(ap) >= (1LL << 31))
     return fail(LL_ERR_UNSUPPORTED, "tensor too large for one call (%lld items)", ll::append_items(ap));
+  if (fp8) return append_stage_and_attend(cache, ap, q, first_frame, n_frames, rope, softmax_scale, out, lse,
+                                          workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
   // the append's frequency tables are built in the kernel's K stages
   const size_t tables = ll::append_smem_bytes(n_frames, cache->H, cache->D, ap.rp.pt);
   // the tables live in the kernel's second Q buffer during the append
@@ -696,6 +793,7 @@ ll_status ll_kv_recache(const ll_kvcache* cache, const void* x, int d_model, con
   p.gamma = gamma;
   p.eps = rms_eps;
   p.M = n_slots * cache->tokens_per_frame;
+  p.B = cache->B;
   p.Din = d_model;
   p.Dout = Dout;
   p.H = cache->H;
@@ -737,18 +835,32 @@ ll_status ll_kv_recache(const ll_kvcache* cache, const void* x, int d_model, con
     return LL_OK;
   });
   if (ast != LL_OK) return ast;
+  // persistent clusters of Dout/256 CTAs (one per column tile), as many as
+  // fit one CTA per SM, each walking every G-th (row block, K or V) tile
+  const int C = Dout / TR::BN;
+  const long long ntiles = 2LL * ((p.M + TR::BM - 1) / TR::BM) * cache->B;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(Dout / TR::BN, (p.M + TR::BM - 1) / TR::BM, 2 * cache->B);
   cfg.blockDim = dim3(TR::THREADS, 1, 1);
   cfg.dynamicSmemBytes = TR::SMEM_BYTES;
   cfg.stream = static_cast<cudaStream_t>(stream);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = Dout / TR::BN;
+  attr[0].val.clusterDim.x = C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  // as many clusters as can be resident at once (a cluster's CTAs must share
+  // one GPC), each walking a contiguous range of tiles
+  int G = 0;
+  cfg.gridDim = dim3(C, 1, 1);
+  if (cudaOccupancyMaxActiveClusters(&G, ll::kv_recache_kernel, &cfg) != cudaSuccess || G < 1) {
+    cudaGetLastError();
+    G = num_sms() / C;
+  }
+  if (G < 1) G = 1;
+  if (G > ntiles) G = static_cast<int>(ntiles);
+  cfg.gridDim = dim3(C, G, 1);
   if (cudaLaunchKernelEx(&cfg, ll::kv_recache_kernel, tmX, tmWk, tmWv, p) != cudaSuccess)
     return check_launch("kv_recache_kernel");
   return check_launch("kv_recache_kernel");

@@ -238,6 +238,10 @@ struct AppendParams {
   int n_sink, n_local;     // cache slots S = n_sink + n_local
   long long first_frame;   // absolute index of the first appended frame
   RopeParams rp;
+  // E4M3 cache only, optional: bf16 rows [B][S*N][H][D] that also receive the
+  // dequantised value (code * scale) of every code written
+  __nv_bfloat16* stage_k;
+  __nv_bfloat16* stage_v;
 };
 
 // Slot of frame f: pinned sink slots first, then a ring over the local slots
@@ -382,19 +386,38 @@ __device__ __forceinline__ void append_store_plain(const AppendParams& p, const 
     }
 }
 
+// bf16 of code * scale for 8 E4M3 codes (the exact code value times the fp32
+// scale, rounded once): the values attention reads from the staging copy.
+__device__ __forceinline__ uint4 decode_chunk8_e4m3_bf16(uint2 codes, float scale) {
+  const uint32_t w[2] = {codes.x, codes.y};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const __nv_fp8x2_storage_t q = static_cast<__nv_fp8x2_storage_t>((w[i] >> (16 * half)) & 0xFFFFu);
+      const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(q, __NV_E4M3);
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+      o[2 * i + half] = pack_bf16(f.x * scale, f.y * scale);
+    }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// The append over blocks blk = 0..nblk-1 of 256 threads (the whole grid of
+// append_kernel, or the append share of the fused E4M3 append + staging).
 template <typename Tin, typename C>
-__global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
+__device__ __forceinline__ void append_blocks(const AppendParams& p, int blk, int nblk) {
   extern __shared__ float s_tab[];      // omega [H][D/2], then cos, sin of the temporal band [F][H][pt][2]
   float* s_omega = s_tab;
   float* s_tcs = s_tab + p.H * (p.D / 2);
   const int cpr = p.D / 8;                        // chunks per (token, head) row
   const int hg = append_heads_per_thread(p.H);    // heads per thread
   const int total = static_cast<int>(append_items(p));  // < 2^31, checked on the host
-  const int stride = gridDim.x * blockDim.x;
+  const int stride = nblk * blockDim.x;
   float kx[kAppendMaxHg][8], vx[kAppendMaxHg][8];
   // the first chunks' loads go out before the tables are built, so the
   // table work overlaps their latency
-  int base = blockIdx.x * blockDim.x;
+  int base = blk * blockDim.x;
   {
     const int idx = base + threadIdx.x;
     append_load<Tin>(p, append_item(p, idx < total ? idx : 0), idx < total, kx, vx);
@@ -428,8 +451,13 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
         const float ks = ka > 0.f ? __fdiv_rn(ka, 448.0f) : 1.0f;
         const float vs = va > 0.f ? __fdiv_rn(va, 448.0f) : 1.0f;
         if (active) {
-          *reinterpret_cast<uint2*>(kc + static_cast<size_t>(k) * p.D) = encode_chunk8_e4m3(kx[k], ks);
-          *reinterpret_cast<uint2*>(vc + static_cast<size_t>(k) * p.D) = encode_chunk8_e4m3(vx[k], vs);
+          const uint2 kq = encode_chunk8_e4m3(kx[k], ks), vq = encode_chunk8_e4m3(vx[k], vs);
+          *reinterpret_cast<uint2*>(kc + static_cast<size_t>(k) * p.D) = kq;
+          *reinterpret_cast<uint2*>(vc + static_cast<size_t>(k) * p.D) = vq;
+          if (p.stage_k != nullptr) {
+            *reinterpret_cast<uint4*>(p.stage_k + it.dst0 + static_cast<size_t>(k) * p.D) = decode_chunk8_e4m3_bf16(kq, ks);
+            *reinterpret_cast<uint4*>(p.stage_v + it.dst0 + static_cast<size_t>(k) * p.D) = decode_chunk8_e4m3_bf16(vq, vs);
+          }
           if (it.c == 0) {
             const size_t srow = it.dst0 / p.D + k;
             p.k_scale[srow] = ks;
@@ -447,6 +475,11 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
   }
 }
 
+template <typename Tin, typename C>
+__global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
+  append_blocks<Tin, C>(p, blockIdx.x, gridDim.x);
+}
+
 // ---------------------------------------------------------------------------
 // E4M3 cache rows -> bf16: value = decode(code) * scale for the first `rows`
 // token rows of every batch entry, K and V (blockIdx.y = 0 / 1). 16 codes
@@ -459,17 +492,19 @@ struct DequantParams {
   int B, rows, batch_rows, H, D;
 };
 
-__global__ void __launch_bounds__(256) dequant_e4m3_kernel(const DequantParams p) {
+// K (isv false) or V rows of every batch entry over blocks blk = 0..nblk-1;
+// rows whose slot (row / N) has its bit set in skip_slots are left alone.
+__device__ __forceinline__ void dequant_blocks(const DequantParams& p, bool isv, int blk, int nblk,
+                                               unsigned long long skip_slots, int N) {
   constexpr int U = 4;  // chunks per thread per pass: their loads are in flight together
-  const bool isv = blockIdx.y != 0;  // K (0) or V (1); selected, not indexed, to keep the params out of local memory
-  const uint8_t* src = isv ? p.src[1] : p.src[0];
+  const uint8_t* src = isv ? p.src[1] : p.src[0];  // selected, not indexed, to keep the params out of local memory
   const float* scale = isv ? p.scale[1] : p.scale[0];
   __nv_bfloat16* dst = isv ? p.dst[1] : p.dst[0];
   const int cpr = p.D / 16;  // 16-code chunks per (token, head) row
   const int per_batch = p.rows * p.H * cpr;
   const int total = p.B * per_batch;
-  const int stride = gridDim.x * blockDim.x;
-  for (int base = blockIdx.x * blockDim.x + threadIdx.x; base < total; base += U * stride) {
+  const int stride = nblk * blockDim.x;
+  for (int base = blk * blockDim.x + threadIdx.x; base < total; base += U * stride) {
     uint4 u[U];
     float sc[U];
     size_t row[U];
@@ -484,7 +519,7 @@ __global__ void __launch_bounds__(256) dequant_e4m3_kernel(const DequantParams p
       row[k] = static_cast<size_t>(b) * p.batch_rows * p.H + th;
       sc[k] = 0.f;
       u[k] = make_uint4(0u, 0u, 0u, 0u);
-      if (idx < total) {
+      if (idx < total && !(skip_slots != 0ull && ((skip_slots >> ((th / p.H) / N)) & 1ull))) {
         sc[k] = scale[row[k]];
         u[k] = *reinterpret_cast<const uint4*>(src + row[k] * p.D + c[k] * 16);
       }
@@ -492,6 +527,10 @@ __global__ void __launch_bounds__(256) dequant_e4m3_kernel(const DequantParams p
 #pragma unroll
     for (int k = 0; k < U; ++k) {
       if (base + k * stride >= total) continue;
+      if (skip_slots != 0ull) {  // skip_slots != 0 only with fewer than 64 slots
+        const int th = static_cast<int>((base + k * stride) % per_batch) / cpr;
+        if ((skip_slots >> ((th / p.H) / N)) & 1ull) continue;
+      }
       const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
       uint32_t o[8];
 #pragma unroll
@@ -508,6 +547,37 @@ __global__ void __launch_bounds__(256) dequant_e4m3_kernel(const DequantParams p
       d[0] = make_uint4(o[0], o[1], o[2], o[3]);
       d[1] = make_uint4(o[4], o[5], o[6], o[7]);
     }
+  }
+}
+
+// blockIdx.y = 0 / 1: K / V rows.
+__global__ void __launch_bounds__(256) dequant_e4m3_kernel(const DequantParams p) {
+  dequant_blocks(p, blockIdx.y != 0, blockIdx.x, gridDim.x, 0ull, 1);
+}
+
+// E4M3 cache: the append of the new frames (RoPE on K, per (token, head)
+// quantisation, codes and scales into their slots, and the dequantised values
+// into the bf16 staging rows) and the dequantisation of every other occupied
+// row into the staging copy, in one launch. Blocks [0, append_blocks) append;
+// the rest are split evenly between the K and V rows of the slots the append
+// does not write (new_slots). The staging rows equal those of
+// ll_kvcache_append followed by the dequantisation pass.
+struct AppendStageParams {
+  AppendParams ap;
+  DequantParams dq;
+  unsigned long long new_slots;  // bit s: slot s is written by the append
+  int append_blocks;
+  int dequant_blocks;            // per K and per V
+};
+
+__global__ void __launch_bounds__(256) append_stage_e4m3_kernel(const AppendStageParams q) {
+  const int blk = blockIdx.x;
+  if (blk < q.append_blocks) {
+    append_blocks<__nv_bfloat16, uint8_t>(q.ap, blk, q.append_blocks);
+  } else {
+    const int d = blk - q.append_blocks;
+    const bool isv = d >= q.dequant_blocks;
+    dequant_blocks(q.dq, isv, isv ? d - q.dequant_blocks : d, q.dequant_blocks, q.new_slots, q.ap.N);
   }
 }
 

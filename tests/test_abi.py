@@ -162,8 +162,13 @@ def _fused(L, cache, rope=None, first=0, nf=1, scale=0.0, ws=1 << 24, ws_bytes=1
 def test_fused_append_attention_validation(L):
     """Every malformed call is rejected on the host, before any launch."""
     fp8 = _cache(dtype=swa.LL_FP8_E4M3, k_scale=1 << 25, v_scale=1 << 26)
-    assert L.ll_append_and_attend_workspace_bytes(ctypes.byref(fp8), 1) == 0
-    assert _fused(L, fp8) == swa.LL_ERR_UNSUPPORTED                 # FP8: the two separate calls
+    # FP8: the attention scratch and the bf16 staging copy, as for attention alone
+    need8 = L.ll_append_and_attend_workspace_bytes(ctypes.byref(fp8), 1)
+    assert need8 == L.ll_sink_window_attention_workspace_bytes(ctypes.byref(fp8), 1) > 0
+    assert _fused(L, fp8, ws_bytes=need8 - 1) == swa.LL_ERR_INVALID_ARG
+    assert _fused(L, fp8, dt=swa.LL_F32) == swa.LL_ERR_INVALID_ARG     # k, v, q are bf16 for an FP8 cache
+    assert _fused(L, _cache(dtype=swa.LL_FP8_E4M3, k_scale=1 << 25, v_scale=1 << 26, D=32),
+                  ws_bytes=1 << 34) == swa.LL_ERR_UNSUPPORTED           # no kernel for D = 32
     assert _fused(L, _cache(D=96)) == swa.LL_ERR_UNSUPPORTED        # no kernel for D = 96
     need = L.ll_append_and_attend_workspace_bytes(ctypes.byref(_cache()), 1)
     assert need > L.ll_sink_window_attention_workspace_bytes(ctypes.byref(_cache()), 1)  # + the barrier word

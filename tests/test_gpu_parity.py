@@ -355,16 +355,18 @@ def test_attention_denoising_passes(chunk):
             assert_parity(np64(out[0]), ref, what=f"frame {f0} pass {ps}")
 
 
-@pytest.mark.parametrize("name", ["wan", "chunk", "tiny", "tiny_d64_b2"])
+@pytest.mark.parametrize("name", ["wan", "chunk", "tiny", "tiny_d64_b2", "wan_fp8", "chunk_fp8", "tiny_d64_b2_fp8"])
 def test_fused_append_attention_matches_separate_calls(name):
     """ll_append_and_attend gives bit-identical outputs, LSE and cache contents
-    to ll_kvcache_append followed by ll_sink_window_attention, from the first
-    frame through the ring wrap."""
+    (codes and scales for an E4M3 cache) to ll_kvcache_append followed by
+    ll_sink_window_attention, from the first frame through the ring wrap."""
+    fp8 = name.endswith("_fp8")
+    base = name[:-4] if fp8 else name
     w = {"wan": W.WAN, "chunk": W.CHUNK, "tiny": W.TINY,
-         "tiny_d64_b2": W.replace(W.TINY, dtype="bf16", name="tiny_d64_b2", B=2)}[name]
+         "tiny_d64_b2": W.replace(W.TINY, dtype="bf16", name="tiny_d64_b2", B=2)}[base]
     rope = rope_of(w)
     c = w.query_frames
-    caches = [swa.KVCache(w.B, w.H, w.D, w.N, w.dtype) for _ in range(2)]
+    caches = [swa.KVCache(w.B, w.H, w.D, w.N, "fp8" if fp8 else w.dtype) for _ in range(2)]
     frames = range(0, 15, c) if w.N < 100 else [0, 3 * c, 11, 12 * c] if c == 1 else [0, 3, 9, 12]
     for f0 in frames:
         q, k, v = (t.cuda() for t in W.qkv_frames(w, 0, f0, c))   # [w.B, c*N, H, D]
@@ -376,6 +378,9 @@ def test_fused_append_attention_matches_separate_calls(name):
         assert torch.equal(o0, o1), f"frame {f0}"
         assert torch.equal(lse[0], lse[1]), f"frame {f0}"
         assert torch.equal(caches[0].k, caches[1].k) and torch.equal(caches[0].v, caches[1].v), f"frame {f0}"
+        if fp8:
+            assert torch.equal(caches[0].k_scale, caches[1].k_scale), f"frame {f0}"
+            assert torch.equal(caches[0].v_scale, caches[1].v_scale), f"frame {f0}"
 
 
 def test_fused_append_attention_stream_parity():
@@ -391,3 +396,19 @@ def test_fused_append_attention_stream_parity():
         rows = sample_rows(q.shape[1], 24, f0)
         ref = so.attend(np64(q[0]), f0, rows=rows)
         assert_parity(np64(out[0])[rows], ref, what=f"fused chunk {f0}")
+
+
+def test_fused_append_attention_fp8_stream_parity():
+    """The fused call over an E4M3 cache against the oracle stream: Wan frames
+    with jitter through the ring wrap, at the FP8 bars."""
+    w = W.replace(W.WAN, sigma_t=0.8, jitter_seed=6, name="wan_jitter")
+    cache = swa.KVCache(w.B, w.H, w.D, w.N, "fp8")
+    rope = rope_of(w)
+    so = StreamOracle(w.H, w.D, w.grid_h, w.grid_w, omega_of(w), w.pairs, w.t_offset)
+    for f0 in range(14):
+        q, k, v = W.qkv_frames(w, 0, f0, 1)
+        out = swa.append_and_attend(cache, k.cuda(), v.cuda(), q.cuda(), f0, rope)
+        so.append(f0, np64(k[0]), np64(v[0]))
+        rows = sample_rows(q.shape[1], 24, f0)
+        ref = so.attend(np64(q[0]), f0, rows=rows)
+        assert_parity(np64(out[0])[rows], ref, max_rel=5e-2, mean_abs=5e-3, what=f"fused fp8 frame {f0}")
