@@ -163,10 +163,13 @@ def max_over_ranks(value: float, dist: bool, device: str = "cuda") -> float:
 class Stream:
     """30 layers of caches and input pools on one GPU."""
 
-    def __init__(self, w: W.Workload, cache_dtype: str, device: str, seed_offset: int = 0, fused: bool = True):
+    def __init__(self, w: W.Workload, cache_dtype: str, device: str, seed_offset: int = 0, fused: bool = True,
+                 fp8_mma: bool = False):
         import sink_window_attention_b200 as swa
         self.swa = swa
-        self.fused = fused  # bf16 / f32 caches: ll_append_and_attend instead of append, then attention
+        self.fused = fused and not fp8_mma  # ll_append_and_attend instead of append, then attention
+        # E4M3 cache read by the FP8 tensor-core attention (ll_sink_window_attention_fp8_mma) after the append
+        self.fp8_mma = fp8_mma and cache_dtype == "fp8"
         self.w = w
         self.device = device
         self.layers = w.layers
@@ -246,6 +249,8 @@ class Stream:
                     attn_events[0].record()
                 if fused:  # append + attention in one kernel
                     swa.append_and_attend(self.caches[l], k, v, q, f, self.rope, out=self.out)
+                elif self.fp8_mma:
+                    swa.sink_window_attention_fp8_mma(q, self.caches[l], f, self.rope, out=self.out)
                 else:
                     swa.sink_window_attention(q, self.caches[l], f, self.rope, out=self.out)
                 launches += self.attention_launches(l)
@@ -266,8 +271,9 @@ class Stream:
 
     def attention_launches(self, layer: int) -> int:
         """Kernel launches of one attention call on this layer's cache (an
-        E4M3 cache: the staging dequantisation (fused: with the append), then
-        the attention kernel)."""
+        E4M3 cache: the staging dequantisation (fused: with the append), or
+        the V-scale pass of the FP8 tensor-core attention, then the attention
+        kernel)."""
         return 2 if self.caches[layer].dtype == "fp8" else 1
 
     def step(self, seg: int, attn_events=None, recache_events=None) -> int:
@@ -374,6 +380,9 @@ def run_ours(args, rank, world, local_rank):
         "hbm_kernels": hbm_kernels(args.cache),
         "fp8_stream": (fp8_stream(args, rank, seed_offset=replica_seed_offset(rank), barrier=barrier, dist=dist)
                        if args.cache == "bf16" and not args.no_fp8_stream else None),
+        "fp8_mma_stream": (fp8_stream(args, rank, seed_offset=replica_seed_offset(rank), barrier=barrier, dist=dist,
+                                      mma=True)
+                           if args.cache == "bf16" and not args.no_fp8_stream else None),
         "gpu_launches": launches,
         "clocks": clk,
     }
@@ -382,13 +391,15 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
-def fp8_stream(args, rank, seed_offset, barrier, dist):
+def fp8_stream(args, rank, seed_offset, barrier, dist, mma: bool = False):
     """The same segment workload over an E4M3 KV cache (per (token, head)
     fp32 scales): `steps` segments after `warmup`, device-timed like the
     main line (max over ranks). Its attention launches time the E4M3 -> bf16
-    staging kernel and the attention kernel together."""
+    staging kernel and the attention kernel together; with `mma`, the
+    V-scale pass and the FP8 tensor-core attention kernel (the append is a
+    launch of its own there)."""
     w = W.replace(W.STREAM_FP8, layers=args.layers)
-    st = Stream(w, "fp8", "cuda", seed_offset=seed_offset)
+    st = Stream(w, "fp8", "cuda", seed_offset=seed_offset, fp8_mma=mma)
     for s in range(args.warmup):
         st.step(s)
     barrier()
@@ -411,8 +422,11 @@ def fp8_stream(args, rank, seed_offset, barrier, dist):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     out = {"value": round(SEGMENT * steps * world / (ms / 1e3), 3), "unit": UNIT, "steps": steps,
            "ms_per_step": round(ms / steps, 3), "kv_cache": "E4M3 codes + fp32 scale per (token, head)",
-           "roofline": {"bound": "tensor", "kernel": "append_stage_e4m3_kernel (append + bf16 staging copy) + "
-                                                      "sink_window_attention_kernel per ll_append_and_attend call",
+           "roofline": {"bound": "tensor",
+                        "kernel": ("scale_max_kernel + sink_window_attention_kernel<E4M3Kv> (kind::f8f6f4) per "
+                                   "ll_sink_window_attention_fp8_mma call; the append is a launch of its own" if mma
+                                   else "append_stage_e4m3_kernel (append + bf16 staging copy) + "
+                                        "sink_window_attention_kernel per ll_append_and_attend call"),
                         "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                         "frac": round(achieved / peak, 4), "avg_launch_us": round(attn_s * 1e6, 2)}}
     del st
@@ -648,7 +662,8 @@ def run_attention_only(args):
     build.build()
     import sink_window_attention_b200 as swa
     w = W.WAN if args.workload == "wan" else W.CHUNK
-    st = Stream(W.replace(w, layers=1, sigma_t=0.8, jitter_seed=4), args.cache, "cuda")
+    st = Stream(W.replace(w, layers=1, sigma_t=0.8, jitter_seed=4), "fp8" if args.cache == "fp8mma" else args.cache,
+                "cuda")
     c = w.query_frames
     q = W.normal((1, c * w.N, w.H, w.D), 99, w.qkv_scale, torch.bfloat16, "cuda")
     out = torch.empty_like(q)
@@ -663,7 +678,10 @@ def run_attention_only(args):
         flush.zero_()
         torch.cuda._sleep(200_000)
         a.record()
-        swa.sink_window_attention(q, st.caches[0], f0, st.rope, out=out)
+        if args.cache == "fp8mma":
+            swa.sink_window_attention_fp8_mma(q, st.caches[0], f0, st.rope, out=out)
+        else:
+            swa.sink_window_attention(q, st.caches[0], f0, st.rope, out=out)
         b.record()
         ev.append((a, b))
     torch.cuda.synchronize()
@@ -801,7 +819,8 @@ def main():
     ap.add_argument("--steps", type=int, default=8)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cache", default="bf16", choices=["bf16", "fp8"])
+    ap.add_argument("--cache", default="bf16", choices=["bf16", "fp8", "fp8mma"],
+                    help="fp8mma (--mode attention): the E4M3 cache read by the FP8 tensor-core attention")
     ap.add_argument("--layers", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--separate", action="store_true", help="append and attention as two calls (bf16 cache)")
@@ -809,6 +828,9 @@ def main():
     ap.add_argument("--mode", default="stream", choices=["stream", "attention", "recache", "append", "rope"])
     ap.add_argument("--workload", default="wan", choices=["wan", "chunk"])
     args = ap.parse_args()
+    if args.cache == "fp8mma" and args.mode != "attention":
+        ap.error("--cache fp8mma times the FP8 tensor-core attention alone (--mode attention); the stream line "
+                 "carries it as fp8_mma_stream")
     if args.mode == "attention":
         print(json.dumps(run_attention_only(args)), flush=True)
         return

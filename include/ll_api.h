@@ -202,6 +202,37 @@ ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvc
                                    size_t workspace_bytes, void* stream);
 
 /*
+ * The same attention over an FP8_E4M3 cache on the FP8 tensor cores (LongLive
+ * model card, abstract: FP8 inference; here it is the KV cache, not the
+ * weights, that is 8-bit). Per 128-row query tile, RoPE(Q) is quantised to
+ * E4M3 with one scale (max|q| / 448); S = Q8 K8^T runs as a kind::f8f6f4
+ * MMA over the cache's codes and is multiplied by the tile's Q scale and each
+ * key's K scale; the softmax weights p are multiplied by each key's V scale
+ * and stored as two E4M3 terms (hi + lo, ~8 significant bits), and
+ * O += P' V8 runs as two kind::f8f6f4 MMAs per key block. The reference
+ * max of each row is lowered by a power of two from the largest V scale of
+ * the head (a pass over the scales before the attention launch) so that P'
+ * stays inside E4M3's range. Results agree with the unquantised attention
+ * to the FP8 tolerance (max error <= 5e-2 max|ref|), not bit for bit with
+ * ll_sink_window_attention over the same cache (which dequantises the cache
+ * into bf16 and computes in bf16).
+ * Arguments, layouts and the other errors as for ll_sink_window_attention;
+ * workspace: at least ll_sink_window_attention_fp8_mma_workspace_bytes(...)
+ * bytes (0 for a cache this entry point does not take).
+ * Errors: LL_ERR_INVALID_ARG for a cache that is not FP8_E4M3 or a q that is
+ * not BF16; LL_ERR_UNSUPPORTED for D != 128 or H not a multiple of 4 (the
+ * scale boxes are 4 heads wide). Two launches: the scale pass, then the
+ * attention.
+ */
+size_t ll_sink_window_attention_fp8_mma_workspace_bytes(const ll_kvcache* cache, int n_query_frames);
+
+ll_status ll_sink_window_attention_fp8_mma(const void* q, ll_dtype q_dtype, const ll_kvcache* cache,
+                                           long long first_frame, int n_query_frames,
+                                           const ll_rope_desc* rope, float softmax_scale,
+                                           void* out, float* lse, void* workspace,
+                                           size_t workspace_bytes, void* stream);
+
+/*
  * ll_kvcache_append of frames first_frame .. first_frame + n_frames - 1
  * followed by ll_sink_window_attention of the same frames as queries, in one
  * kernel: each CTA writes its share of the new frames' K/V into their slots

@@ -28,7 +28,8 @@ EXPORTED = (
     "ll_kvcache_append", "ll_sink_window_attention_workspace_bytes", "ll_sink_window_attention",
     "ll_kv_recache_workspace_bytes", "ll_kv_recache", "ll_sink_window_attention_noalloc",
     "ll_append_and_attend_workspace_bytes", "ll_append_and_attend", "ll_phase_coherence",
-    "ll_selftest_bounded_waits",
+    "ll_selftest_bounded_waits", "ll_sink_window_attention_fp8_mma_workspace_bytes",
+    "ll_sink_window_attention_fp8_mma",
 )
 NOALLOC_SCRATCH_BYTES = 48 * 1024 * 1024
 
@@ -75,6 +76,9 @@ def lib() -> ctypes.CDLL:
         L.ll_sink_window_attention_workspace_bytes.restype = sz
         L.ll_sink_window_attention.argtypes = [vp, i, cp, ll_, i, rp, f, vp, vp, vp, sz, vp]
         L.ll_sink_window_attention_noalloc.argtypes = [vp, i, cp, ll_, i, rp, f, vp, vp, vp]
+        L.ll_sink_window_attention_fp8_mma_workspace_bytes.argtypes = [cp, i]
+        L.ll_sink_window_attention_fp8_mma_workspace_bytes.restype = sz
+        L.ll_sink_window_attention_fp8_mma.argtypes = [vp, i, cp, ll_, i, rp, f, vp, vp, vp, sz, vp]
         L.ll_kv_recache_workspace_bytes.argtypes = [cp, i, i]
         L.ll_kv_recache_workspace_bytes.restype = sz
         L.ll_kv_recache.argtypes = [cp, vp, i, vp, vp, vp, f, ctypes.POINTER(ll_), i, rp, vp, sz, vp]
@@ -294,6 +298,29 @@ def sink_window_attention(q: torch.Tensor, cache: KVCache, first_frame: int, rop
     _check(lib().ll_sink_window_attention(_ptr(q), _dtype_code(q.dtype), ctypes.byref(_cache_c(cache)), first_frame, F,
                                           _rope_ref(rope), float(softmax_scale), _ptr(out), _ptr(lse),
                                           _ptr(workspace), ws_bytes, _stream(stream)))
+    return out
+
+
+def attention_fp8_mma_workspace_bytes(cache: KVCache, n_query_frames: int) -> int:
+    return int(lib().ll_sink_window_attention_fp8_mma_workspace_bytes(ctypes.byref(cache.to_c()), n_query_frames))
+
+
+def sink_window_attention_fp8_mma(q: torch.Tensor, cache: KVCache, first_frame: int, rope: Optional[Rope],
+                                  softmax_scale: float = 0.0, out: Optional[torch.Tensor] = None,
+                                  lse: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                                  stream=None) -> torch.Tensor:
+    """Attention over an E4M3 cache on the FP8 tensor cores (ll_sink_window_attention_fp8_mma)."""
+    F = _check_shape(cache, q, "q")
+    if out is None:
+        out = torch.empty_like(q)
+    _expect(out, q.shape, q.dtype, "out")
+    _expect(lse, (cache.B, cache.H, q.shape[1]), torch.float32, "lse")
+    if workspace is None:
+        workspace = workspace_for(max(attention_fp8_mma_workspace_bytes(cache, F), 256), q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().ll_sink_window_attention_fp8_mma(_ptr(q), _dtype_code(q.dtype), ctypes.byref(_cache_c(cache)),
+                                                  first_frame, F, _rope_ref(rope), float(softmax_scale), _ptr(out),
+                                                  _ptr(lse), _ptr(workspace), ws_bytes, _stream(stream)))
     return out
 
 

@@ -186,6 +186,25 @@ ll_status encode_rows_map(CUtensorMap* map, const void* base, CUtensorMapDataTyp
   return LL_OK;
 }
 
+// 3D map over an E4M3 cache's fp32 scales [B][batch_rows][H]: dims (H, rows,
+// B), box (4 heads, box_rows, 1), 16 bytes wide, so its x coordinate (the
+// first head) is always a multiple of 4; heads >= H and rows >= `rows` read as
+// 0. The row stride H * 4 bytes must be a multiple of 16 (H % 4 == 0).
+ll_status encode_scale_map(CUtensorMap* map, const void* base, int H, long long rows, long long batch_rows, int B,
+                           int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(LL_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint64_t dims[3] = {(cuuint64_t)H, (cuuint64_t)rows, (cuuint64_t)B};
+  const cuuint64_t strides[2] = {(cuuint64_t)H * 4, (cuuint64_t)batch_rows * H * 4};
+  const cuuint32_t box[3] = {4u, (cuuint32_t)box_rows, 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LL_ERR_CUDA, "cuTensorMapEncodeTiled (scales) failed (%d)", (int)r);
+  return LL_OK;
+}
+
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Workspace of one attention call: per-unit arrival counters, then
@@ -209,17 +228,26 @@ ll_status launch_attention(ll::AttnParams p, const ll_kvcache* c, long long S, v
     return fail(LL_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu required", ws_bytes, need);
   p.counters = static_cast<int*>(workspace);
   p.partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(p.units * sizeof(int)));
-  CUtensorMap tmK, tmV;
-  const CUtensorMapDataType dt = TR::ES == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  CUtensorMap tmQ, tmK, tmV, tmKS, tmVS;
+  // Q (and O) are bf16 in the E4M3 variant; its K and V are 1-byte codes
+  const CUtensorMapDataType dq =
+      TR::FP8 || TR::ES == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const CUtensorMapDataType dkv = TR::FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : dq;
+  const int qes = TR::FP8 ? 2 : TR::ES;
   const long long batch_rows = S * c->tokens_per_frame;
-  CUtensorMap tmQ;
-  ll_status st = encode_rows_map(&tmQ, p.q, dt, TR::ES, TR::D, c->H, p.Tq, p.Tq, c->B, TR::BM);
+  ll_status st = encode_rows_map(&tmQ, p.q, dq, qes, TR::D, c->H, p.Tq, p.Tq, c->B, TR::BM);
   if (st != LL_OK) return st;
-  st = encode_rows_map(&tmK, c->k, dt, TR::ES, TR::D, c->H, p.Nk, batch_rows, c->B, TR::BN);
+  st = encode_rows_map(&tmK, c->k, dkv, TR::ES, TR::D, c->H, p.Nk, batch_rows, c->B, TR::BN);
   if (st != LL_OK) return st;
-  st = encode_rows_map(&tmV, c->v, dt, TR::ES, TR::D, c->H, p.Nk, batch_rows, c->B, TR::BN,
-                       TR::ES == 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B);
+  st = encode_rows_map(&tmV, c->v, dkv, TR::ES, TR::D, c->H, p.Nk, batch_rows, c->B, TR::BN,
+                       TR::ES <= 2 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B);
   if (st != LL_OK) return st;
+  tmKS = tmK;  // read only by the E4M3 variant
+  tmVS = tmK;
+  if constexpr (TR::FP8) {
+    if ((st = encode_scale_map(&tmKS, c->k_scale, c->H, p.Nk, batch_rows, c->B, TR::BN)) != LL_OK) return st;
+    if ((st = encode_scale_map(&tmVS, c->v_scale, c->H, p.Nk, batch_rows, c->B, TR::BN)) != LL_OK) return st;
+  }
   auto kern = ll::sink_window_attention_kernel<TR>;
   static std::atomic<unsigned long long> attr_set{0};
   st = once_per_device(attr_set, [&]() -> ll_status {
@@ -231,7 +259,7 @@ ll_status launch_attention(ll::AttnParams p, const ll_kvcache* c, long long S, v
   if (cudaMemsetAsync(p.counters, 0, p.units * sizeof(int), stream) != cudaSuccess)
     return check_launch("cudaMemsetAsync(attention counters)");
   if (!cooperative) {
-    kern<<<p.grid, TR::THREADS, TR::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
+    kern<<<p.grid, TR::THREADS, TR::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmKS, tmVS, p);
     return check_launch("sink_window_attention_kernel");
   }
   // fused append: the CTAs meet at a grid barrier, so they must all be
@@ -246,7 +274,7 @@ ll_status launch_attention(ll::AttnParams p, const ll_kvcache* c, long long S, v
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, tmQ, tmK, tmV, p) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, kern, tmQ, tmK, tmV, tmKS, tmVS, p) != cudaSuccess)
     return check_launch("sink_window_attention_kernel (cooperative, fused append)");
   return check_launch("sink_window_attention_kernel (cooperative, fused append)");
 }
@@ -533,6 +561,78 @@ ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvc
   if (f32 && cache->D == 64)
     return launch_attention<ll::AttnTraits<64, float>>(p, cache, S, workspace, workspace_bytes, s);
   return fail(LL_ERR_UNSUPPORTED, "attention supports D = 64 or 128 (bf16) and D = 64 (f32); got D = %d", cache->D);
+}
+
+size_t ll_sink_window_attention_fp8_mma_workspace_bytes(const ll_kvcache* cache, int n_query_frames) {
+  if (cache == nullptr || n_query_frames < 1 || cache->tokens_per_frame < 1 || cache->H < 1 || cache->B < 1 ||
+      cache->dtype != LL_FP8_E4M3 || cache->D != 128)
+    return 0;
+  const int units = ((n_query_frames * cache->tokens_per_frame + 127) / 128) * cache->H * cache->B;
+  return align256(attention_workspace<ll::AttnTraits<128, ll::E4M3Kv>>(units)) +
+         align256(static_cast<size_t>(cache->B) * cache->H * sizeof(float));  // + the V-scale maxima
+}
+
+ll_status ll_sink_window_attention_fp8_mma(const void* q, ll_dtype q_dtype, const ll_kvcache* cache,
+                                           long long first_frame, int n_query_frames, const ll_rope_desc* rope,
+                                           float softmax_scale, void* out, float* lse, void* workspace,
+                                           size_t workspace_bytes, void* stream) {
+  g_last_error.clear();
+  ll_status st = check_cache(cache);
+  if (st != LL_OK) return st;
+  if (cache->dtype != LL_FP8_E4M3)
+    return fail(LL_ERR_INVALID_ARG, "ll_sink_window_attention_fp8_mma reads an FP8_E4M3 cache");
+  if (cache->D != 128 || cache->H % 4 != 0)
+    return fail(LL_ERR_UNSUPPORTED, "the FP8 tensor-core attention needs D = 128 and H a multiple of 4 (D = %d, H = %d)",
+                cache->D, cache->H);
+  if (q_dtype != LL_BF16) return fail(LL_ERR_INVALID_ARG, "q dtype must be BF16");
+  if (q == nullptr || out == nullptr) return fail(LL_ERR_INVALID_ARG, "q and out must be non-NULL");
+  if (!aligned16(q) || !aligned16(out)) return fail(LL_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
+  if (!aligned4(lse)) return fail(LL_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+  if (first_frame < 0) return fail(LL_ERR_INVALID_ARG, "first_frame must be >= 0");
+  if (n_query_frames < 1 || n_query_frames > cache->n_local)
+    return fail(LL_ERR_INVALID_ARG, "n_query_frames = %d must lie in [1, n_local = %d]", n_query_frames,
+                cache->n_local);
+  if (!(softmax_scale >= 0.f) || !std::isfinite(softmax_scale))
+    return fail(LL_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  const size_t need = ll_sink_window_attention_fp8_mma_workspace_bytes(cache, n_query_frames);
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(LL_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu required", workspace_bytes, need);
+  if (!aligned16(workspace)) return fail(LL_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  if ((st = check_grid(rope, cache->tokens_per_frame)) != LL_OK) return st;
+  const long long S = cache->n_sink + cache->n_local;
+  const long long last = first_frame + n_query_frames - 1;
+  const long long valid_slots = last + 1 < S ? last + 1 : S;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ll::AttnParams p{};
+  if ((st = make_rope(rope, cache->H, cache->D, first_frame, &p.rp)) != LL_OK) return st;  // before any launch
+  // the largest V scale of each (batch, head) over the valid keys
+  const int units = ((n_query_frames * cache->tokens_per_frame + 127) / 128) * cache->H * cache->B;
+  float* v_scale_max = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                                align256(attention_workspace<ll::AttnTraits<128, ll::E4M3Kv>>(units)));
+  if (cudaMemsetAsync(v_scale_max, 0, static_cast<size_t>(cache->B) * cache->H * sizeof(float), s) != cudaSuccess)
+    return check_launch("cudaMemsetAsync(V scale maxima)");
+  ll::ScaleMaxParams sp{};
+  sp.scale = cache->v_scale;
+  sp.out = reinterpret_cast<unsigned int*>(v_scale_max);
+  sp.rows = static_cast<int>(valid_slots * cache->tokens_per_frame);
+  sp.batch_rows = static_cast<int>(S * cache->tokens_per_frame);
+  sp.H = cache->H;
+  const int per = 256 / cache->H;
+  const long long want = (sp.rows + per - 1) / per;
+  const dim3 grid(static_cast<unsigned>(want < num_sms() ? want : num_sms()), static_cast<unsigned>(cache->B));
+  ll::scale_max_kernel<<<grid, 256, 0, s>>>(sp);
+  if ((st = check_launch("scale_max_kernel")) != LL_OK) return st;
+  p.q = q;
+  p.out = out;
+  p.lse = lse;
+  p.B = cache->B;
+  p.H = cache->H;
+  p.Tq = n_query_frames * cache->tokens_per_frame;
+  p.Nk = static_cast<int>(valid_slots * cache->tokens_per_frame);
+  p.softmax_scale = softmax_scale;
+  p.N = cache->tokens_per_frame;
+  p.v_scale_max = v_scale_max;
+  return launch_attention<ll::AttnTraits<128, ll::E4M3Kv>>(p, cache, S, workspace, workspace_bytes, s);
 }
 
 }  // extern "C"

@@ -38,34 +38,47 @@
 //    (warp-collective) only run under warp-uniform conditions.
 #pragma once
 
+#include <type_traits>
+
 #include "ll_common.cuh"
 #include "ll_rope_append.cuh"
 
 namespace ll {
 
+// Marks the attention variant over an E4M3 cache on the FP8 tensor cores:
+// the bf16 Q tile is quantised to E4M3 (one scale per tile) in shared memory,
+// K and V arrive as E4M3 codes with their per-(token, head) scales, and
+// S = Q K^T and O += P' V run as kind::f8f6f4 MMAs.
+struct E4M3Kv {};
+
 template <int D_, typename T_>
 struct AttnTraits {
-  using T = T_;
+  static constexpr bool FP8 = std::is_same<T_, E4M3Kv>::value;
+  using T = typename std::conditional<FP8, __nv_bfloat16, T_>::type;  // Q and O
   static constexpr int D = D_;
-  static constexpr int ES = sizeof(T);
+  static constexpr int ES = FP8 ? 1 : static_cast<int>(sizeof(T));  // bytes per MMA operand element
   static constexpr int BM = 128;                    // query rows per tile (TMEM lanes)
   static constexpr int BN = 128;                    // keys per KV tile
-  static constexpr int ROWB = D * ES;               // bytes of one Q/K/V row
+  static constexpr int ROWB = D * ES;               // bytes of one Q/K/V operand row
   static constexpr int NB = ROWB / 128;             // 128-byte column blocks per row
   static constexpr int ELEMS_PER_BLOCK = 128 / ES;  // elements of D per column block
-  static constexpr int Q_BYTES = BM * ROWB;
+  static constexpr int Q_BYTES = BM * ROWB;         // one Q operand tile
+  static constexpr int QSTG_BYTES = FP8 ? BM * D * 2 : 0;  // bf16 tile that the E4M3 Q is quantised from
   static constexpr int KV_BYTES = BN * ROWB;
+  static constexpr int SC_BYTES = FP8 ? 2 * BN * 16 : 0;  // K and V scale boxes ([BN][4 heads] fp32) per V stage
+  static constexpr int VSTAGE_BYTES = KV_BYTES + SC_BYTES;
   static constexpr int QK_STEPS = ROWB / 32;        // MMAs per S tile (32 bytes of K each)
-  static constexpr int PV_STEPS = BN * ES / 32;     // MMAs per P V (8 bf16 / 16 tf32)
+  static constexpr int PV_STEPS = BN * ES / 32;     // MMAs per P V (8 bf16 / 16 tf32 / 4 e4m3)
   static constexpr int MMA_K = 32 / ES;             // reduction elements per MMA
-  static constexpr int FMT = (ES == 2) ? 1 : 2;     // bf16 / tf32
+  static constexpr int FMT = FP8 ? 0 : (ES == 2) ? 1 : 2;  // e4m3 / bf16 / tf32
   static constexpr int QST = 2;                     // Q buffers
   static constexpr int CTRL_BYTES = 2048;
-  static constexpr int STAGE_BUDGET = 232448 - CTRL_BYTES - 1024 - QST * Q_BYTES;
+  static constexpr int STAGE_BUDGET = 232448 - CTRL_BYTES - 1024 - QST * Q_BYTES - QSTG_BYTES;
   static constexpr int STAGES = STAGE_BUDGET / KV_BYTES;
-  static constexpr int KST = STAGES >= 8 ? 4 : (STAGES + 1) / 2;
-  static constexpr int VST = STAGES >= 8 ? 4 : STAGES - KST;
-  static constexpr int SMEM_BYTES = CTRL_BYTES + 1024 + QST * Q_BYTES + (KST + VST) * KV_BYTES;
+  static constexpr int KST = FP8 ? 4 : STAGES >= 8 ? 4 : (STAGES + 1) / 2;
+  static constexpr int VST = FP8 ? 4 : STAGES >= 8 ? 4 : STAGES - KST;
+  static constexpr int SMEM_BYTES =
+      CTRL_BYTES + 1024 + QST * Q_BYTES + QSTG_BYTES + KST * KV_BYTES + VST * VSTAGE_BYTES;
   static constexpr int TMEM_COLS = 512;
   static constexpr int S_COL0 = 0, O_COL0 = 2 * BN;  // S_w at w*BN, O_w at O_COL0 + w*D
   static constexpr int THREADS = 384;
@@ -82,6 +95,8 @@ struct AttnTraits {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(O_COL0 + 2 * D <= TMEM_COLS, "TMEM budget");
   static_assert(NB >= 1 && ROWB % 128 == 0, "rows must be whole 128-byte blocks");
+  static_assert(!FP8 || D == 128, "the E4M3 variant is written for D = 128 (one 128-byte row)");
+  static_assert(VSTAGE_BYTES % 1024 == 0 && QSTG_BYTES % 1024 == 0, "1024-byte aligned buffers");
 };
 
 struct AttnParams {
@@ -106,6 +121,10 @@ struct AttnParams {
   unsigned int gen;                // generation tag of this launch in the barrier word
   unsigned long long* grid_bar;    // [generation:32 | arrivals:32]
   AppendParams ap;                 // the append (input dtype = cache dtype = T)
+  // E4M3 variant: the largest V scale of each (batch, head) over the valid
+  // keys ([B][H], from a pass before the launch); it fixes the power-of-two
+  // shift of the reference max that keeps P' = p * scale_v inside E4M3's range
+  const float* v_scale_max;
 };
 
 // A piece: key tiles [j0, j0 + n) of unit u.
@@ -168,6 +187,61 @@ __device__ __forceinline__ void rope_q_tile_inplace(uint8_t* sQ, const AttnParam
   fence_proxy_async_smem();  // the generic-proxy writes are read by the tensor core
 }
 
+// E4M3 variant: quantise the bf16 Q tile in `stage` (RoPE already applied;
+// 128-byte swizzled K-major, D/64 column blocks) into the E4M3 operand tile
+// `q8` (one 128-byte block per row, same swizzle) with one scale per tile:
+// scale = max|q| / 448 (1 for a zero tile), codes = RNE(q / scale) saturated.
+// Threads tid 0..nthreads-1 synchronise on named barrier `bar`; every thread
+// passes both barriers whatever `active` says (a thread whose wait gave up
+// passes inactive), so the barrier counts always match. `amax_word` is a
+// shared word this call may overwrite.
+template <class TR>
+__device__ __forceinline__ void quantize_q_tile(const uint8_t* stage, uint8_t* q8, float* scale_out,
+                                                unsigned int* amax_word, int tid, int nthreads, int bar, bool active) {
+  constexpr int BM = TR::BM, D = TR::D;
+  if (tid == 0) *amax_word = 0u;
+  asm volatile("bar.sync %0, %1;" ::"r"(bar), "r"(nthreads) : "memory");
+  float amax = 0.f;
+  for (int g = active ? tid : BM * (D / 8); g < BM * (D / 8); g += nthreads) {
+    const int r = g / (D / 8), e8 = g - r * (D / 8);
+    const uint4 v = *reinterpret_cast<const uint4*>(stage + (e8 >> 3) * (BM * 128) + sw128_offset(r, e8 & 7));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+      amax = fmax3(amax, fabsf(f.x), fabsf(f.y));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((tid & 31) == 0) atomicMax(amax_word, __float_as_uint(amax));  // non-negative floats order as integers
+  asm volatile("bar.sync %0, %1;" ::"r"(bar), "r"(nthreads) : "memory");
+  const float tmax = __uint_as_float(*amax_word);
+  const float sc = tmax > 0.f ? tmax / 448.0f : 1.0f;
+  const float inv = 1.0f / sc;
+  for (int g = active ? tid : BM * (D / 16); g < BM * (D / 16); g += nthreads) {
+    const int r = g / (D / 16), c = g - r * (D / 16);  // output chunk c: elements 16c .. 16c + 15
+    uint32_t out[4];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int e8 = 2 * c + half;
+      const uint4 v = *reinterpret_cast<const uint4*>(stage + (e8 >> 3) * (BM * 128) + sw128_offset(r, e8 & 7));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[2 * i]));
+        const float2 f1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[2 * i + 1]));
+        const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(f0.x * inv, f0.y * inv), __NV_SATFINITE, __NV_E4M3);
+        const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(f1.x * inv, f1.y * inv), __NV_SATFINITE, __NV_E4M3);
+        out[2 * half + i] = lo | (hi << 16);
+      }
+    }
+    *reinterpret_cast<uint4*>(q8 + sw128_offset(r, c)) = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+  if (tid == 0) *scale_out = sc;
+  fence_proxy_async_smem();  // the generic-proxy writes are read by the tensor core
+}
+
 // TMA copy of the Q tile of unit u into a Q buffer (NB column blocks of 128
 // bytes x BM rows; rows past Tq read as zeros). One thread.
 template <class TR>
@@ -183,15 +257,19 @@ __device__ __forceinline__ void tma_q_tile(uint8_t* dst, const CUtensorMap* tmQ,
 template <class TR>
 __global__ void __launch_bounds__(384, 1)
     sink_window_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                                 const __grid_constant__ CUtensorMap tmV, const AttnParams p) {
+                                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKS,
+                                 const __grid_constant__ CUtensorMap tmVS, const AttnParams p) {
   using T = typename TR::T;
+  // the Q tile as loaded: bf16 staging for the E4M3 variant, else the operand itself
+  using QTR = typename std::conditional<TR::FP8, AttnTraits<TR::D, __nv_bfloat16>, TR>::type;
   constexpr int BM = TR::BM, BN = TR::BN, D = TR::D, KST = TR::KST, VST = TR::VST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                              // [QST][Q_BYTES]
-  uint8_t* sK = sQ + TR::QST * TR::Q_BYTES;        // [KST][KV_BYTES]
-  uint8_t* sV = sK + KST * TR::KV_BYTES;           // [VST][KV_BYTES]
-  uint8_t* ctrl = sV + VST * TR::KV_BYTES;
+  uint8_t* sQs = sQ + TR::QST * TR::Q_BYTES;       // [QSTG_BYTES] bf16 Q tile (E4M3 variant)
+  uint8_t* sK = sQs + TR::QSTG_BYTES;              // [KST][KV_BYTES]
+  uint8_t* sV = sK + KST * TR::KV_BYTES;           // [VST][VSTAGE_BYTES]: V tile (+ K and V scale boxes)
+  uint8_t* ctrl = sV + VST * TR::VSTAGE_BYTES;
   uint64_t* k_full = reinterpret_cast<uint64_t*>(ctrl);
   uint64_t* k_empty = k_full + KST;
   uint64_t* v_full = k_empty + KST;
@@ -212,6 +290,9 @@ __global__ void __launch_bounds__(384, 1)
   float* s_mB = reinterpret_cast<float*>(ctrl + 384);      // [128]
   float* s_lB = s_mB + BM;                                 // [128]
   float* s_omega = reinterpret_cast<float*>(ctrl + 1408);  // [2][D/2]: one head per Q buffer
+  float* s_qscale = reinterpret_cast<float*>(ctrl + 1920);  // [2] E4M3 variant: scale of each Q buffer
+  unsigned int* s_qamax = reinterpret_cast<unsigned int*>(ctrl + 1928);
+  static_assert(1408 + 2 * (D / 2) * 4 <= 1920 && 1932 <= TR::CTRL_BYTES, "control block layout");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = blockIdx.x;
@@ -271,8 +352,8 @@ __global__ void __launch_bounds__(384, 1)
     long long it0 = it_begin;
     Piece pc0;
     next_piece(it0, pc0);
-    if (threadIdx.x == 64) tma_q_tile<TR>(sQ, &tmQ, &q_tma[0], p, pc0.u);
-    if (p.fuse_append) {
+    if (threadIdx.x == 64) tma_q_tile<QTR>(TR::FP8 ? sQs : sQ, &tmQ, &q_tma[0], p, pc0.u);
+    if (!TR::FP8 && p.fuse_append) {
       // This CTA's contiguous share of the new frames' tokens (all batch
       // entries): their K and V rows come into the K/V stage buffers (which
       // TMA fills only after the barrier) by bulk copies, K is rotated in
@@ -348,16 +429,23 @@ __global__ void __launch_bounds__(384, 1)
             });
           bulk_store_commit_wait();  // complete before the rows are reused or the barrier is passed
         }
-        __syncthreads();
+        if (r0 + R < t1) __syncthreads();  // the next round reuses the buffers
       }
-      // the cache rows written here are read by TMA (async proxy) after the
-      // barrier, and TMA refills the buffers that held the rows and tables
-      asm volatile("fence.proxy.async.global;" ::: "memory");
-      fence_proxy_async_smem();
-      __threadfence();
-      __syncthreads();
-      if (threadIdx.x == 0) grid_barrier(p.grid_bar, p.gen, static_cast<unsigned int>(p.grid), s_abort);
-      __syncthreads();
+      // Every thread's shared-memory writes (rows, tables) were fenced for the
+      // async proxy before the last round's bulk stores, and thread 0 alone
+      // wrote global memory (those stores, complete). Thread 0 fences them for
+      // the other CTAs' TMA reads and meets those CTAs at the grid barrier; it
+      // then issues every K/V load into the stage buffers that held the rows.
+      // The Q loader, which refills the buffer that held the tables, passed
+      // the last round's block barrier after every access to them. The other
+      // warps go on meanwhile: the first Q tile's RoPE needs nothing from the
+      // append.
+      if (threadIdx.x == 0) {
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __threadfence();
+        grid_barrier(p.grid_bar, p.gen, static_cast<unsigned int>(p.grid), s_abort);
+      }
+      __syncwarp();  // warp 0 reconverges before its setmaxnreg
     }
     if (warp >= 2) {
       const int tid = threadIdx.x - 64;  // 0..319
@@ -365,9 +453,13 @@ __global__ void __launch_bounds__(384, 1)
         for (int j = tid; j < D / 2; j += 320) s_omega[j] = omega_of(p.rp, (pc0.u / p.q_tiles) % p.H, j);
       asm volatile("bar.sync 4, 320;" ::: "memory");
       const bool landed = mbar_wait(&q_tma[0], 0, s_abort);
-      if (landed && p.rp.enabled) rope_q_tile_inplace<TR>(sQ, p, s_omega, pc0.u, tid, 320);
+      if (landed && p.rp.enabled) rope_q_tile_inplace<QTR>(TR::FP8 ? sQs : sQ, p, s_omega, pc0.u, tid, 320);
       if (!landed && tid == 0) mbar_wait_teardown(&q_tma[0], 0);  // the copy must land before the CTA exits
       asm volatile("bar.sync 4, 320;" ::: "memory");
+      if constexpr (TR::FP8) {
+        quantize_q_tile<TR>(sQs, sQ, &s_qscale[0], s_qamax, tid, 320, 4, landed);
+        asm volatile("bar.sync 4, 320;" ::: "memory");
+      }
       if (tid == 0) mbar_arrive(&q_full[0]);
     }
   }
@@ -380,6 +472,10 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
+      if constexpr (TR::FP8) {
+        tma_prefetch_desc(&tmKS);
+        tma_prefetch_desc(&tmVS);
+      }
       if (p.fuse_append) asm volatile("fence.proxy.async.global;" ::: "memory");  // see the append above
       // K and V walk the same tile sequence with cursors of their own; each
       // is loaded as soon as its ring has a free stage, so K runs ahead of V
@@ -411,11 +507,19 @@ __global__ void __launch_bounds__(384, 1)
         if (hv && mbar_test(smem_addr(&v_empty[vc % VST]), ((vc / VST) & 1) ^ 1)) {
           const int st = vc % VST;
           const int h = (pv.u / p.q_tiles) % p.H, b = pv.u / (p.q_tiles * p.H);
-          mbar_expect_tx(&v_full[st], TR::KV_BYTES);
+          mbar_expect_tx(&v_full[st], TR::VSTAGE_BYTES);
 #pragma unroll
           for (int blk = 0; blk < TR::NB; ++blk)
-            tma_load_4d(sV + st * TR::KV_BYTES + blk * (BN * 128), &tmV, &v_full[st], blk * TR::ELEMS_PER_BLOCK, h,
-                        (pv.j0 + iv) * BN, b);
+            tma_load_4d(sV + st * TR::VSTAGE_BYTES + blk * (BN * 128), &tmV, &v_full[st], blk * TR::ELEMS_PER_BLOCK,
+                        h, (pv.j0 + iv) * BN, b);
+          if constexpr (TR::FP8) {
+            // the tile's K and V scales ride with the V tile: [BN keys][4 heads]
+            // fp32 boxes from head h rounded down to a multiple of 4 (so that
+            // the box's x coordinate is 16-byte aligned)
+            uint8_t* sc = sV + st * TR::VSTAGE_BYTES + TR::KV_BYTES;
+            tma_load_3d(sc, &tmKS, &v_full[st], h & ~3, (pv.j0 + iv) * BN, b);
+            tma_load_3d(sc + BN * 16, &tmVS, &v_full[st], h & ~3, (pv.j0 + iv) * BN, b);
+          }
           ++vc;
           if (++iv == pv.n) {
             iv = 0;
@@ -459,7 +563,7 @@ __global__ void __launch_bounds__(384, 1)
       // descriptor words of every buffer, computed once; an MMA then only adds
       // a constant to the low word
       const DescWords dQ = desc_words(aQ, 16, 1024, 2), dK = desc_words(aK, 16, 1024, 2);
-      const DescWords dV = TR::ES == 2 ? desc_words(aV, BN * 128, 1024, 2) : desc_words(aV, BN * 128, 512, 1);
+      const DescWords dV = TR::ES <= 2 ? desc_words(aV, BN * 128, 1024, 2) : desc_words(aV, BN * 128, 512, 1);
       auto issue_s = [&](int w, int qb) -> bool {
         const int st = kc % KST;
         if (!mbar_wait(&k_full[st], (kc / KST) & 1, s_abort)) return false;
@@ -472,7 +576,8 @@ __global__ void __launch_bounds__(384, 1)
           const uint32_t offk = (k >> 2) * (BN * 128) + (k & 3) * 32;
           const uint64_t da = desc_at(dQ, qoff + off);
           const uint64_t db = desc_at(dK, koff + offk);
-          if constexpr (TR::ES == 2) mma_bf16_ss(d, da, db, idS, k > 0 ? 1u : 0u);
+          if constexpr (TR::FP8) mma_f8_ss(d, da, db, idS, k > 0 ? 1u : 0u);
+          else if constexpr (TR::ES == 2) mma_bf16_ss(d, da, db, idS, k > 0 ? 1u : 0u);
           else mma_tf32_ss(d, da, db, idS, k > 0 ? 1u : 0u);
         }
         mma_commit(&s_full[w]);
@@ -484,11 +589,15 @@ __global__ void __launch_bounds__(384, 1)
         const int st = vc % VST;
         const uint32_t d = tbase + TR::O_COL0 + w * D;
         const uint32_t pa = tbase + TR::S_COL0 + w * BN;  // P_w aliases S_w
-        const uint32_t voff = st * TR::KV_BYTES;
+        const uint32_t voff = st * TR::VSTAGE_BYTES;
 #pragma unroll
         for (int k = 0; k < TR::PV_STEPS; ++k) {
           const uint64_t db = desc_at(dV, voff + k * TR::MMA_K * 128);
-          if constexpr (TR::ES == 2) mma_bf16_ts(d, pa + k * 8, db, idO, (acc || k > 0) ? 1u : 0u);
+          if constexpr (TR::FP8) {  // P' = hi + lo: two MMAs per K step
+            mma_f8_ts(d, pa + k * 8, db, idO, (acc || k > 0) ? 1u : 0u);
+            mma_f8_ts(d, pa + TR::BN / 4 + k * 8, db, idO, 1u);
+          }
+          else if constexpr (TR::ES == 2) mma_bf16_ts(d, pa + k * 8, db, idO, (acc || k > 0) ? 1u : 0u);
           else mma_tf32_ts(d, pa + k * 8, db, idO, (acc || k > 0) ? 1u : 0u);
         }
         mma_commit(&o_done[w]);
@@ -528,15 +637,22 @@ __global__ void __launch_bounds__(384, 1)
       const int qb = pidx & 1;
       const int h = (pc.u / p.q_tiles) % p.H;
       bool ok = mbar_wait(&q_empty[qb], ((pidx >> 1) & 1) ^ 1, s_abort);
-      if (ok && tid == 0) tma_q_tile<TR>(sQ + qb * TR::Q_BYTES, &tmQ, &q_tma[qb], p, pc.u);
+      if (ok && tid == 0) tma_q_tile<QTR>(TR::FP8 ? sQs : sQ + qb * TR::Q_BYTES, &tmQ, &q_tma[qb], p, pc.u);
       float* om = s_omega + qb * (D / 2);
       if (ok && p.rp.enabled)
         for (int j = tid; j < D / 2; j += 64) om[j] = omega_of(p.rp, h, j);
       asm volatile("bar.sync 2, 64;" ::: "memory");
+      bool q_ok = false;
       if (ok) {
         const bool landed = mbar_wait(&q_tma[qb], (pidx >> 1) & 1, s_abort);
-        if (landed && p.rp.enabled) rope_q_tile_inplace<TR>(sQ + qb * TR::Q_BYTES, p, om, pc.u, tid, 64);
+        if (landed && p.rp.enabled)
+          rope_q_tile_inplace<QTR>(TR::FP8 ? sQs : sQ + qb * TR::Q_BYTES, p, om, pc.u, tid, 64);
         if (!landed && tid == 0) mbar_wait_teardown(&q_tma[qb], (pidx >> 1) & 1);  // let the copy land
+        q_ok = landed;
+      }
+      if constexpr (TR::FP8) {
+        asm volatile("bar.sync 2, 64;" ::: "memory");  // the RoPE writes are visible
+        quantize_q_tile<TR>(sQs, sQ + qb * TR::Q_BYTES, &s_qscale[qb], s_qamax, tid, 64, 2, q_ok);
       }
       asm volatile("bar.sync 2, 64;" ::: "memory");
       if (tid == 0) mbar_arrive(&q_full[qb]);
@@ -558,14 +674,39 @@ __global__ void __launch_bounds__(384, 1)
     long long it = it_begin;
     Piece pc;
     int cnt = 0, pidx = 0;
+    int vbase = 0;  // V tiles of the earlier pieces (E4M3 variant: the stage that holds a tile's scales)
     bool ok = true;
     while (next_piece(it, pc)) {
       float m_run = -INFINITY, l_run = 0.f;
       int mine = 0;
+      // E4M3 variant: S = scale_q * scale_k * (Q8 K8^T); the tile's Q scale
+      // folds into the exponent factor, the per-key K scale multiplies S.
+      // P' = p * scale_v (per key) is what the tensor core multiplies with
+      // V8; the reference max is lowered by kshift so that P' stays below 448.
+      float sqsl2 = sl2, kshift = 0.f;
+      int hq = 0;
+      if constexpr (TR::FP8) {
+        const int qb = pidx & 1;
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&q_full[qb], (pidx >> 1) & 1, s_abort));  // Q scale written
+        sqsl2 = s_qscale[qb] * sl2;
+        const int hh = (pc.u / p.q_tiles) % p.H, bb = pc.u / (p.q_tiles * p.H);
+        const float svm = p.v_scale_max[bb * p.H + hh];
+        kshift = svm > 0.f ? fminf(fmaxf(floorf(log2f(1.75f / svm)), -64.f), 64.f) : 0.f;
+        hq = hh & 3;
+      }
       for (int i = wg; i < pc.n; i += 2, ++mine) {
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], cnt & 1, s_abort));
         if (!ok) continue;
         tc_fence_after();
+        const float* skb = nullptr;  // [BN][4] K scales of this tile (E4M3 variant)
+        const float* svb = nullptr;  // [BN][4] V scales
+        if constexpr (TR::FP8) {
+          const int vidx = vbase + i, vs = vidx % VST;
+          ok = __all_sync(0xffffffffu, mbar_wait(&v_full[vs], (vidx / VST) & 1, s_abort));
+          if (!ok) continue;
+          skb = reinterpret_cast<const float*>(sV + vs * TR::VSTAGE_BYTES + TR::KV_BYTES) + hq;
+          svb = skb + BN * 4;
+        }
         uint32_t sr[BN / 32][32];
         constexpr int HC = BN / 64;  // chunks of 32 columns per half
         const int kv_valid = p.Nk - (pc.j0 + i) * BN;
@@ -587,6 +728,12 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
             for (int c = HC; c < 2 * HC; ++c) tmem_load_wait(sr[c]);
           }
+          if constexpr (TR::FP8) {
+#pragma unroll
+            for (int c = hf * HC; c < (hf + 1) * HC; ++c)
+#pragma unroll
+              for (int e = 0; e < 32; ++e) sr[c][e] = __float_as_uint(__uint_as_float(sr[c][e]) * skb[(c * 32 + e) * 4]);
+          }
           if (kv_valid < BN) {
 #pragma unroll
             for (int c = hf * HC; c < (hf + 1) * HC; ++c)
@@ -601,11 +748,11 @@ __global__ void __launch_bounds__(384, 1)
               mx8[e & 7] = fmax3(mx8[e & 7], __uint_as_float(sr[c][2 * e]), __uint_as_float(sr[c][2 * e + 1]));
         }
         const float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
-        const float m_new = mx * sl2;
+        const float m_new = mx * sqsl2;
         float m_use = m_run;
         bool rescale = false;
-        if (m_new > m_run + 8.0f) {
-          m_use = m_new;
+        if (m_new > m_run + kshift + 8.0f) {  // m_run is the reference: the row max minus kshift
+          m_use = m_new - kshift;
           rescale = (mine > 0);
         }
         // S_i complete implies this warpgroup's previous P V (issued before it) is complete
@@ -626,10 +773,11 @@ __global__ void __launch_bounds__(384, 1)
         // p = 2^(s * scale * log2(e) - m) on pairs: the argument with one packed
         // FMA, the exponential on the MUFU unit, the running sum in 4 packed
         // partial sums
-        const uint64_t sl2x2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m_use, -m_use);
+        const uint64_t sl2x2 = f2_pack(sqsl2, sqsl2), negm2 = f2_pack(-m_use, -m_use);
         uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
+          uint32_t plo[8];  // E4M3 variant: the lo terms of this chunk's P'
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const uint64_t x2 =
@@ -638,14 +786,33 @@ __global__ void __launch_bounds__(384, 1)
             f2_unpack(x2, x0, x1);
             const float a = ex2(x0), a2 = ex2(x1);
             ls2[e & 3] = f2_add(ls2[e & 3], f2_pack(a, a2));
-            if constexpr (TR::ES == 2) {
+            if constexpr (TR::FP8) {
+              // P' = p * scale_v as two E4M3 terms, hi + lo (lo: the fp16
+              // residual), ~8 significant bits in all; four keys per 32-bit
+              // word, key 4w in the low byte
+              const __half2 ph = __floats2half2_rn(a * svb[(c * 32 + 2 * e) * 4], a2 * svb[(c * 32 + 2 * e + 1) * 4]);
+              const uint32_t hi = __nv_cvt_halfraw2_to_fp8x2(ph, __NV_SATFINITE, __NV_E4M3);
+              const __half2 hih = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(hi), __NV_E4M3);
+              const uint32_t lo = __nv_cvt_halfraw2_to_fp8x2(__hsub2(ph, hih), __NV_SATFINITE, __NV_E4M3);
+              if (e & 1) {
+                sr[c][e >> 1] |= hi << 16;
+                plo[e >> 1] |= lo << 16;
+              } else {
+                sr[c][e >> 1] = hi;
+                plo[e >> 1] = lo;
+              }
+            } else if constexpr (TR::ES == 2) {
               sr[c][e] = pack_bf16(a, a2);  // packed in place: slot e is free once 2e, 2e+1 were read
             } else {
               sr[c][2 * e] = __float_as_uint(a);
               sr[c][2 * e + 1] = __float_as_uint(a2);
             }
           }
-          if constexpr (TR::ES == 2) tmem_store16(tS + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[c][0]));
+          if constexpr (TR::FP8) {  // hi terms in columns [0, 32), lo terms in [32, 64)
+            tmem_store8(tS + c * 8, *reinterpret_cast<uint32_t(*)[8]>(&sr[c][0]));
+            tmem_store8(tS + BN / 4 + c * 8, plo);
+          }
+          else if constexpr (TR::ES == 2) tmem_store16(tS + c * 16, *reinterpret_cast<uint32_t(*)[16]>(&sr[c][0]));
           else tmem_store32(tS + c * 32, sr[c]);
         }
         {
@@ -802,6 +969,7 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
+      vbase += pc.n;
       ++pidx;
     }
   }

@@ -317,6 +317,13 @@ __device__ __forceinline__ void tmem_store32(uint32_t taddr, const uint32_t (&r)
       "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+__device__ __forceinline__ void tmem_store8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8};\n\t" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_store16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -368,6 +375,27 @@ __device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// kind::f8f6f4 with both operands E4M3 (the instruction descriptor's A and B
+// format fields select the 8-bit type); A from shared memory or from tensor
+// memory (four K elements per 32-bit column).
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -426,8 +454,9 @@ __device__ __forceinline__ uint64_t desc_mn_sw128_atom32(uint32_t saddr, uint32_
   return d;
 }
 
-// Instruction descriptor, dense kind::f16 / kind::tf32, fp32 accumulator.
-// fmt: 0 = f16, 1 = bf16, 2 = tf32 (both operands share it).
+// Instruction descriptor, dense kind::f16 / kind::tf32 / kind::f8f6f4, fp32
+// accumulator. fmt: kind::f16: 0 = f16, 1 = bf16; kind::tf32: 2;
+// kind::f8f6f4: 0 = E4M3 (both operands share it).
 __host__ __device__ constexpr uint32_t idesc_dense(int M, int N, int fmt, bool a_mn_major, bool b_mn_major) {
   return (1u << 4)                                   // D format: f32
          | (static_cast<uint32_t>(fmt) << 7)         // A format

@@ -481,6 +481,36 @@ __global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
 }
 
 // ---------------------------------------------------------------------------
+// Largest scale of each (batch, head) over the first `rows` tokens of an E4M3
+// cache's scale array [B][batch_rows][H]: out[b * H + h], zeroed before the
+// launch (scales are positive, so their bits order as unsigned integers and
+// atomicMax on the bits is the float maximum). Grid (x: row blocks, y: batch);
+// H <= kMaxHeads.
+// ---------------------------------------------------------------------------
+struct ScaleMaxParams {
+  const float* scale;
+  unsigned int* out;
+  int rows, batch_rows, H;
+};
+
+__global__ void __launch_bounds__(256) scale_max_kernel(const ScaleMaxParams p) {
+  __shared__ unsigned int smax[kMaxHeads];
+  for (int i = threadIdx.x; i < p.H; i += blockDim.x) smax[i] = 0u;
+  __syncthreads();
+  const int b = blockIdx.y;
+  const int per = blockDim.x / p.H;  // tokens a pass of the block reads
+  const int h = threadIdx.x % p.H, r0 = threadIdx.x / p.H;
+  if (r0 < per) {
+    float m = 0.f;
+    for (int r = blockIdx.x * per + r0; r < p.rows; r += gridDim.x * per)
+      m = fmaxf(m, p.scale[(static_cast<size_t>(b) * p.batch_rows + r) * p.H + h]);
+    atomicMax(&smax[h], __float_as_uint(m));
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < p.H; i += blockDim.x) atomicMax(&p.out[b * p.H + i], smax[i]);
+}
+
+// ---------------------------------------------------------------------------
 // E4M3 cache rows -> bf16: value = decode(code) * scale for the first `rows`
 // token rows of every batch entry, K and V (blockIdx.y = 0 / 1). 16 codes
 // (16 bytes) per thread.

@@ -106,6 +106,43 @@ def test_attention_validation(L):
     assert "workspace" in swa.last_error()
 
 
+def test_fp8_mma_attention_validation(L):
+    """The FP8 tensor-core entry point takes only an E4M3 cache with D = 128 and
+    H a multiple of 4, a BF16 q, and the rest as ll_sink_window_attention;
+    every case fails on the host before the scale pass is launched."""
+    fp8 = dict(dtype=swa.LL_FP8_E4M3, k_scale=1 << 22, v_scale=1 << 23)
+
+    def call(cache, rope=None, first=0, nq=1, scale=0.0, ws=1 << 24, ws_bytes=1 << 40, q=1 << 20, qdt=swa.LL_BF16):
+        return L.ll_sink_window_attention_fp8_mma(q, qdt, ctypes.byref(cache), first, nq,
+                                                  ctypes.byref(rope) if rope is not None else None, scale,
+                                                  1 << 21, None, ws, ws_bytes, None)
+
+    need = L.ll_sink_window_attention_fp8_mma_workspace_bytes(ctypes.byref(_cache(**fp8)), 1)
+    assert need > 0
+    # larger than the bf16 kernel's scratch for the same frames: + the [B][H] V-scale maxima
+    assert need >= L.ll_sink_window_attention_workspace_bytes(ctypes.byref(_cache()), 1) + 12 * 4
+    assert L.ll_sink_window_attention_fp8_mma_workspace_bytes(ctypes.byref(_cache()), 1) == 0
+    assert L.ll_sink_window_attention_fp8_mma_workspace_bytes(ctypes.byref(_cache(D=64, **fp8)), 1) == 0
+    cases = [
+        (dict(cache=_cache()), swa.LL_ERR_INVALID_ARG, "FP8_E4M3"),
+        (dict(cache=_cache(dtype=swa.LL_FP8_E4M3)), swa.LL_ERR_INVALID_ARG, "k_scale"),
+        (dict(cache=_cache(D=64, **fp8)), swa.LL_ERR_UNSUPPORTED, "D = 128"),
+        (dict(cache=_cache(H=6, **fp8)), swa.LL_ERR_UNSUPPORTED, "multiple of 4"),
+        (dict(cache=_cache(**fp8), qdt=swa.LL_F32), swa.LL_ERR_INVALID_ARG, "BF16"),
+        (dict(cache=_cache(**fp8), nq=10), swa.LL_ERR_INVALID_ARG, "n_query_frames"),
+        (dict(cache=_cache(**fp8), first=-1), swa.LL_ERR_INVALID_ARG, "first_frame"),
+        (dict(cache=_cache(**fp8), scale=float("nan")), swa.LL_ERR_INVALID_ARG, "softmax_scale"),
+        (dict(cache=_cache(**fp8), q=(1 << 20) + 2), swa.LL_ERR_INVALID_ARG, "aligned"),
+        (dict(cache=_cache(**fp8), ws_bytes=16), swa.LL_ERR_INVALID_ARG, "workspace"),
+        (dict(cache=_cache(**fp8), rope=_rope(pairs_t=10)), swa.LL_ERR_INVALID_ARG, "sum to D/2"),
+        (dict(cache=_cache(**fp8), rope=_rope(grid_w=51)), swa.LL_ERR_INVALID_ARG, "does not match"),
+    ]
+    for kw, want, msg in cases:
+        st = call(**kw)
+        assert st == want, (kw, st, swa.last_error())
+        assert msg in swa.last_error(), (kw, swa.last_error())
+
+
 def test_append_and_rope_validation(L):
     k = v = 1 << 20
     rc = ctypes.byref(_rope())
@@ -150,6 +187,7 @@ def test_recache_validation(L):
     fp8 = _cache(dtype=swa.LL_FP8_E4M3, k_scale=(1 << 22) + 1, v_scale=1 << 23)
     assert call(cache=fp8) == swa.LL_ERR_INVALID_ARG                      # scales written as floats
     assert "4-byte" in swa.last_error()
+
 
 
 def _fused(L, cache, rope=None, first=0, nf=1, scale=0.0, ws=1 << 24, ws_bytes=1 << 30, k=1 << 20, v=1 << 21,

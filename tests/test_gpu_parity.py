@@ -148,7 +148,7 @@ def test_append_fp8_codes_and_scales():
 # ---------------------------------------------------------------------------- attention
 def run_stream(w: W.Workload, frames, layer=0, rows_per_step=48, q_scale=1.0, check_lse=True, dtype=None,
                B=None, mean_abs=1e-3, lse_rel=1e-3, max_rel=1e-2, scale=None, k_scale=None, no_rope=False,
-               t_scale=1.0, lse_mean=5e-3, n_sink=3, n_local=9):
+               t_scale=1.0, lse_mean=5e-3, n_sink=3, n_local=9, attend=None):
     """Append + attend frame by frame (or chunk by chunk); compare sampled rows
     (all rows when the step is small) with the oracle stream."""
     B = B or w.B
@@ -174,7 +174,7 @@ def run_stream(w: W.Workload, frames, layer=0, rows_per_step=48, q_scale=1.0, ch
             k = (k.float() * k_scale(f0)).to(k.dtype)
         swa.kvcache_append(cache, k.cuda(), v.cuda(), f0, rope)
         lse = torch.empty(B, w.H, q.shape[1], device="cuda", dtype=torch.float32)
-        out = swa.sink_window_attention(q.cuda(), cache, f0, rope, lse=lse, softmax_scale=scale or 0.0)
+        out = (attend or swa.sink_window_attention)(q.cuda(), cache, f0, rope, lse=lse, softmax_scale=scale or 0.0)
         Tq = q.shape[1]
         rows = np.arange(Tq) if Tq <= 256 else sample_rows(Tq, rows_per_step, f0)
         for b in range(B):
@@ -292,6 +292,26 @@ def test_attention_fp8_cache(name, frames):
     unquantised fp64 reference, max|err| <= 5e-2 * max|ref|."""
     w = W.WORKLOADS[name]
     run_stream(w, frames, dtype="fp8", rows_per_step=24, mean_abs=5e-3, lse_rel=5e-3, max_rel=5e-2)
+
+
+@pytest.mark.parametrize("name,frames", [("wan", range(14)), ("chunk", range(0, 15, 3))])
+def test_attention_fp8_mma(name, frames):
+    """E4M3 cache on the FP8 tensor cores (ll_sink_window_attention_fp8_mma:
+    Q quantised per tile, S and P' V as kind::f8f6f4 MMAs over the cache's
+    codes) through warm-up, the ring wrap and steady state, against the
+    unquantised fp64 reference at the FP8 bars."""
+    w = W.WORKLOADS[name]
+    run_stream(w, frames, dtype="fp8", rows_per_step=24, mean_abs=5e-3, lse_rel=5e-3, max_rel=5e-2,
+               attend=swa.sink_window_attention_fp8_mma)
+
+
+def test_attention_fp8_mma_small_batch2():
+    """The FP8 tensor-core attention on two batch entries of a small chunk
+    stream (4 heads, 6x10 grid: 60 tokens per frame, so every key count is a
+    ragged multiple of the 128-key tile), every output row checked."""
+    w = W.replace(W.CHUNK, name="chunk_small_fp8", H=4, grid_h=6, grid_w=10, t_offset=500)
+    run_stream(w, range(0, 18, 3), dtype="fp8", B=2, mean_abs=5e-3, lse_rel=5e-3, max_rel=5e-2,
+               attend=swa.sink_window_attention_fp8_mma)
 
 
 def test_attention_fp8_cache_d64_staged():
