@@ -337,10 +337,28 @@ ll_status append_stage_and_attend(const ll_kvcache* cache, const ll::AppendParam
   dp.batch_rows = static_cast<int>(S * cache->tokens_per_frame);
   dp.H = cache->H;
   dp.D = cache->D;
-  for (int i = 0; i < n_frames; ++i) {
-    int slot = 0;
-    ll_slot_of_frame(first_frame + i, cache->n_sink, cache->n_local, &slot);
-    q8.new_slots |= 1ull << slot;
+  dp.cshift = cache->D == 128 ? 3 : 2;
+  // the appended frames' slots as runs of consecutive slots (a ring wrap
+  // splits them; a sink and a local frame can join): their (token, head) rows
+  // are written by the append blocks and skipped by the staging blocks
+  {
+    bool is_new[ll::kMaxSlots] = {};
+    for (int i = 0; i < n_frames; ++i) {
+      int slot = 0;
+      ll_slot_of_frame(first_frame + i, cache->n_sink, cache->n_local, &slot);
+      is_new[slot] = true;
+    }
+    const int per_slot = cache->tokens_per_frame * cache->H;
+    for (int sl = 0; sl < S;) {
+      if (!is_new[sl]) { ++sl; continue; }
+      int e = sl;
+      while (e < S && is_new[e]) ++e;
+      if (dp.nskip == 3) return fail(LL_ERR_UNSUPPORTED, "the appended frames' slots form more than 3 runs");
+      dp.skip_lo[dp.nskip] = sl * per_slot;
+      dp.skip_hi[dp.nskip] = e * per_slot;
+      ++dp.nskip;
+      sl = e;
+    }
   }
   const long long threads = ll::append_items(ap);
   const long long want_a = (threads + 255) / 256;
@@ -533,6 +551,7 @@ ll_status ll_sink_window_attention(const void* q, ll_dtype q_dtype, const ll_kvc
     dp.batch_rows = static_cast<int>(S * cache->tokens_per_frame);
     dp.H = cache->H;
     dp.D = cache->D;
+    dp.cshift = cache->D == 128 ? 3 : 2;
     const long long chunks = static_cast<long long>(dp.B) * dp.rows * dp.H * (dp.D / 16);
     const long long want = (chunks + 255) / 256;
     const dim3 grid(static_cast<unsigned>(want < 8LL * num_sms() ? want : 8LL * num_sms()), 2);

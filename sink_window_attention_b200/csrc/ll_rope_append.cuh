@@ -520,69 +520,71 @@ struct DequantParams {
   const float* scale[2];
   __nv_bfloat16* dst[2];
   int B, rows, batch_rows, H, D;
+  int cshift;                   // log2(D / 16): 16-code chunks per (token, head) row
+  int nskip;                    // rows left alone: (token, head) rows [skip_lo[i], skip_hi[i]) of every batch entry
+  int skip_lo[3], skip_hi[3];
 };
 
-// K (isv false) or V rows of every batch entry over blocks blk = 0..nblk-1;
-// rows whose slot (row / N) has its bit set in skip_slots are left alone.
-__device__ __forceinline__ void dequant_blocks(const DequantParams& p, bool isv, int blk, int nblk,
-                                               unsigned long long skip_slots, int N) {
-  constexpr int U = 4;  // chunks per thread per pass: their loads are in flight together
+// K (isv false) or V rows of every batch entry over blocks blk = 0..nblk-1.
+// The first `rows` token rows of a batch entry are contiguous ([rows][H][D]
+// codes, [rows][H] scales), so chunk i of a batch entry (16 codes) starts at
+// code 16 i and belongs to (token, head) row i >> cshift: no division in the
+// index arithmetic.
+// U: chunks per thread per pass, their loads in flight together.
+template <int U>
+__device__ __forceinline__ void dequant_blocks(const DequantParams& p, bool isv, int blk, int nblk) {
   const uint8_t* src = isv ? p.src[1] : p.src[0];  // selected, not indexed, to keep the params out of local memory
   const float* scale = isv ? p.scale[1] : p.scale[0];
   __nv_bfloat16* dst = isv ? p.dst[1] : p.dst[0];
-  const int cpr = p.D / 16;  // 16-code chunks per (token, head) row
-  const int per_batch = p.rows * p.H * cpr;
-  const int total = p.B * per_batch;
+  const int per_batch = (p.rows * p.H) << p.cshift;
   const int stride = nblk * blockDim.x;
-  for (int base = blk * blockDim.x + threadIdx.x; base < total; base += U * stride) {
-    uint4 u[U];
-    float sc[U];
-    size_t row[U];
-    int c[U];
+  for (int b = 0; b < p.B; ++b) {
+    const size_t row0 = static_cast<size_t>(b) * p.batch_rows * p.H;  // first (token, head) row of the entry
+    const uint4* srcb = reinterpret_cast<const uint4*>(src + row0 * p.D);
+    const float* scb = scale + row0;
+    uint4* dstb = reinterpret_cast<uint4*>(dst + row0 * p.D);
+    for (int base = blk * blockDim.x + threadIdx.x; base < per_batch; base += U * stride) {
+      uint4 u[U];
+      float sc[U];
+      bool go[U];
 #pragma unroll
-    for (int k = 0; k < U; ++k) {
-      const int idx = base + k * stride;
-      const int b = idx / per_batch;
-      const int r = idx - b * per_batch;  // (token * H + h) * cpr + c within the batch entry
-      const int th = r / cpr;             // token-head row
-      c[k] = r - th * cpr;
-      row[k] = static_cast<size_t>(b) * p.batch_rows * p.H + th;
-      sc[k] = 0.f;
-      u[k] = make_uint4(0u, 0u, 0u, 0u);
-      if (idx < total && !(skip_slots != 0ull && ((skip_slots >> ((th / p.H) / N)) & 1ull))) {
-        sc[k] = scale[row[k]];
-        u[k] = *reinterpret_cast<const uint4*>(src + row[k] * p.D + c[k] * 16);
+      for (int k = 0; k < U; ++k) {
+        const int idx = base + k * stride;
+        const int th = idx >> p.cshift;
+        bool g = idx < per_batch;
+#pragma unroll
+        for (int i = 0; i < 3; ++i)  // constant indices keep the params out of local memory
+          if (i < p.nskip) g = g && !(th >= p.skip_lo[i] && th < p.skip_hi[i]);
+        go[k] = g;
+        sc[k] = g ? scb[th] : 0.f;
+        u[k] = g ? srcb[idx] : make_uint4(0u, 0u, 0u, 0u);
       }
-    }
 #pragma unroll
-    for (int k = 0; k < U; ++k) {
-      if (base + k * stride >= total) continue;
-      if (skip_slots != 0ull) {  // skip_slots != 0 only with fewer than 64 slots
-        const int th = static_cast<int>((base + k * stride) % per_batch) / cpr;
-        if ((skip_slots >> ((th / p.H) / N)) & 1ull) continue;
-      }
-      const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
-      uint32_t o[8];
+      for (int k = 0; k < U; ++k) {
+        if (!go[k]) continue;
+        const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+        uint32_t o[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 4; ++i) {
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const __nv_fp8x2_storage_t q = static_cast<__nv_fp8x2_storage_t>((w[i] >> (16 * half)) & 0xFFFFu);
-          const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(q, __NV_E4M3);
-          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
-          o[2 * i + half] = pack_bf16(f.x * sc[k], f.y * sc[k]);
+          for (int half = 0; half < 2; ++half) {
+            const __nv_fp8x2_storage_t q = static_cast<__nv_fp8x2_storage_t>((w[i] >> (16 * half)) & 0xFFFFu);
+            const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(q, __NV_E4M3);
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+            o[2 * i + half] = pack_bf16(f.x * sc[k], f.y * sc[k]);
+          }
         }
+        const int idx = base + k * stride;
+        dstb[2 * idx] = make_uint4(o[0], o[1], o[2], o[3]);
+        dstb[2 * idx + 1] = make_uint4(o[4], o[5], o[6], o[7]);
       }
-      uint4* d = reinterpret_cast<uint4*>(dst + row[k] * p.D + c[k] * 16);
-      d[0] = make_uint4(o[0], o[1], o[2], o[3]);
-      d[1] = make_uint4(o[4], o[5], o[6], o[7]);
     }
   }
 }
 
 // blockIdx.y = 0 / 1: K / V rows.
 __global__ void __launch_bounds__(256) dequant_e4m3_kernel(const DequantParams p) {
-  dequant_blocks(p, blockIdx.y != 0, blockIdx.x, gridDim.x, 0ull, 1);
+  dequant_blocks<4>(p, blockIdx.y != 0, blockIdx.x, gridDim.x);
 }
 
 // E4M3 cache: the append of the new frames (RoPE on K, per (token, head)
@@ -590,12 +592,11 @@ __global__ void __launch_bounds__(256) dequant_e4m3_kernel(const DequantParams p
 // into the bf16 staging rows) and the dequantisation of every other occupied
 // row into the staging copy, in one launch. Blocks [0, append_blocks) append;
 // the rest are split evenly between the K and V rows of the slots the append
-// does not write (new_slots). The staging rows equal those of
+// does not write (dq's skip ranges). The staging rows equal those of
 // ll_kvcache_append followed by the dequantisation pass.
 struct AppendStageParams {
   AppendParams ap;
-  DequantParams dq;
-  unsigned long long new_slots;  // bit s: slot s is written by the append
+  DequantParams dq;              // with the rows of the appended frames' slots skipped
   int append_blocks;
   int dequant_blocks;            // per K and per V
 };
@@ -607,7 +608,8 @@ __global__ void __launch_bounds__(256) append_stage_e4m3_kernel(const AppendStag
   } else {
     const int d = blk - q.append_blocks;
     const bool isv = d >= q.dequant_blocks;
-    dequant_blocks(q.dq, isv, isv ? d - q.dequant_blocks : d, q.dequant_blocks, q.new_slots, q.ap.N);
+    // the append's register allocation leaves few blocks per SM: more loads in flight per thread
+    dequant_blocks<8>(q.dq, isv, isv ? d - q.dequant_blocks : d, q.dequant_blocks);
   }
 }
 
