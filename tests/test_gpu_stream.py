@@ -7,8 +7,9 @@ cache; "Frame Sink" and "Short-Window Attention": every frame attends to the
 3 sink frames plus the most recent local frames.
 
 * The benchmark's own stream driver (bench.Stream: per frame and layer the
-  fused append + attention for a bf16 cache, append then attention for an
-  E4M3 cache; at a switch the recache of every layer) runs frames 12..52 of
+  fused append + attention for a bf16 cache, the append with the bf16
+  staging copy then attention for an E4M3 cache, or the append then the FP8
+  tensor-core attention; at a switch the recache of every layer) runs frames 12..52 of
   several layers with a prompt switch before frame 40; sampled query rows of
   every layer at frames 28..52 are compared with one oracle stream per layer
   fed the same pooled inputs and the same hidden states and projections.
@@ -65,11 +66,12 @@ def oracle_stream(w: W.Workload) -> StreamOracle:
     return StreamOracle(w.H, w.D, w.grid_h, w.grid_w, om, w.pairs, w.t_offset)
 
 
-@pytest.mark.parametrize("cache", ["bf16", "fp8"])
+@pytest.mark.parametrize("cache", ["bf16", "fp8", "fp8mma"])
 def test_bench_stream_across_prompt_switch(cache):
     layers, switch, last, check_from = 3, 40, 53, 28
     w = W.replace(W.STREAM if cache == "bf16" else W.STREAM_FP8, layers=layers)
-    st = bench.Stream(w, cache, "cuda")           # caches filled with frames 0..11 of the pools
+    # fp8mma: the E4M3 cache read by the FP8 tensor-core attention (fp8_mma_stream of the bench line)
+    st = bench.Stream(w, "fp8" if cache == "fp8mma" else cache, "cuda", fp8_mma=cache == "fp8mma")
     N, P = w.N, bench.POOL
     rows = sample_rows(N, 8, 0)
     rows_dev = torch.as_tensor(rows, device="cuda")
@@ -86,7 +88,7 @@ def test_bench_stream_across_prompt_switch(cache):
     assert swa.device_error() == 0
     assert sorted(got) == [(f, l) for f in range(check_from, last) for l in range(layers)]
 
-    bars = dict(max_rel=5e-2, mean_abs=5e-3) if cache == "fp8" else {}
+    bars = dict(max_rel=5e-2, mean_abs=5e-3) if cache != "bf16" else {}
     # the hidden states are in slot order: slot s holds the frame the oracle's
     # own slot map puts there after frame switch - 1
     held = owin.slot_frames(switch - 1)
