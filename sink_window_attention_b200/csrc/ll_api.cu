@@ -432,14 +432,14 @@ ll_status ll_rope_apply(void* x, ll_dtype dtype, int B, int n_frames, int H, int
   p.D = D;
   const long long chunks = static_cast<long long>(B) * n_frames * p.N * H * (D / 8);
   if (chunks >= (1LL << 31)) return fail(LL_ERR_UNSUPPORTED, "tensor too large for one call (%lld chunks)", chunks);
-  const long long want = (chunks + 255) / 256;
-  const int grid = static_cast<int>(want < 8LL * num_sms() ? want : 8LL * num_sms());
-  const size_t smem = static_cast<size_t>(H) * (D / 2) * sizeof(float);
+  if (H * (D / 8) > 1024) return fail(LL_ERR_UNSUPPORTED, "H * D / 8 = %d exceeds 1024", H * (D / 8));
+  const long long rows = static_cast<long long>(B) * n_frames * p.N;
+  const int grid = static_cast<int>((rows + ll::kRopeTokens - 1) / ll::kRopeTokens);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dtype == LL_BF16)
-    ll::rope_apply_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(p);
+    ll::rope_apply_kernel<__nv_bfloat16><<<grid, H * (D / 8), 0, s>>>(p);
   else
-    ll::rope_apply_kernel<float><<<grid, 256, smem, s>>>(p);
+    ll::rope_apply_kernel<float><<<grid, H * (D / 8), 0, s>>>(p);
   return check_launch("rope_apply_kernel");
 }
 

@@ -193,32 +193,53 @@ struct RopeApplyParams {
   RopeParams rp;
 };
 
+// One thread per (head, 8-element chunk) of a token row (blockDim = H * D/8),
+// kRopeTokens token rows per block: a thread's head and pairs, hence its 4
+// frequencies, are the same for every row it rotates, so they are evaluated
+// once per thread; the rows' positions once per row; the loads of all rows
+// are issued before any rotation.
+constexpr int kRopeTokens = 4;
+
 template <typename T>
-__global__ void __launch_bounds__(256) rope_apply_kernel(const RopeApplyParams p) {
-  extern __shared__ float s_omega[];  // [H][D/2]
-  const int P = p.D / 2;
-  build_omega(s_omega, p.rp, 0, p.H, P);
-  __syncthreads();
-  const int cpr = p.D / 8;  // chunks per (token, head) row
-  const int total = p.B * p.F * p.N * p.H * cpr;  // < 2^31, checked on the host
-  const int FN = p.F * p.N;
-  T* x = static_cast<T*>(p.x);
+__global__ void __launch_bounds__(1024) rope_apply_kernel(const RopeApplyParams p) {
+  __shared__ float s_pos[kRopeTokens][3];  // temporal, row and column position of each token row
+  const int cpr = p.D / 8;
+  const int h = threadIdx.x / cpr, c = threadIdx.x - h * cpr;
+  const int rows = p.B * p.F * p.N;
+  const int r0 = blockIdx.x * kRopeTokens;
+  const int nt = min(kRopeTokens, rows - r0);
+  if (threadIdx.x < nt) {
+    const int tok = (r0 + threadIdx.x) % (p.F * p.N);
+    const int fi = tok / p.N, n = tok - fi * p.N;
+    const int r = n / p.rp.grid_w;
+    s_pos[threadIdx.x][0] = temporal_pos(p.rp, fi);
+    s_pos[threadIdx.x][1] = static_cast<float>(r);
+    s_pos[threadIdx.x][2] = static_cast<float>(n - r * p.rp.grid_w);
+  }
   const int pth = p.rp.pt + p.rp.ph;
-  for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < total; idx += gridDim.x * blockDim.x) {
-    const int row = idx / cpr;
-    const int c = idx - row * cpr;
-    const int bt = row / p.H;
-    const int h = row - bt * p.H;
-    const int tok = bt % FN;
-    const int fi = tok / p.N;
-    const int n = tok - fi * p.N;
-    const int r = n / p.rp.grid_w, col = n - r * p.rp.grid_w;
-    float v[8];
-    T* ptr = x + static_cast<size_t>(row) * p.D + c * 8;
-    load_chunk8<T>(ptr, v);
-    rotate_chunk8(v, c * 4, temporal_pos(p.rp, fi), static_cast<float>(r),
-                  static_cast<float>(col), s_omega + h * P, p.rp.pt, pth);
-    store_chunk8<T>(ptr, v);
+  float om[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) om[q] = omega_of(p.rp, h, c * 4 + q);
+  T* x = static_cast<T*>(p.x) + (static_cast<size_t>(r0) * p.H + h) * p.D + c * 8;
+  float v[kRopeTokens][8];
+#pragma unroll
+  for (int k = 0; k < kRopeTokens; ++k)
+    if (k < nt) load_chunk8<T>(x + static_cast<size_t>(k) * p.H * p.D, v[k]);
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < kRopeTokens; ++k) {
+    if (k >= nt) break;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int j = c * 4 + q;
+      const float pos = j < p.rp.pt ? s_pos[k][0] : (j < pth ? s_pos[k][1] : s_pos[k][2]);
+      float sn, cs;
+      sincos_reduced(pos * om[q], sn, cs);
+      const float a = v[k][2 * q], b = v[k][2 * q + 1];
+      v[k][2 * q] = a * cs - b * sn;
+      v[k][2 * q + 1] = a * sn + b * cs;
+    }
+    store_chunk8<T>(x + static_cast<size_t>(k) * p.H * p.D, v[k]);
   }
 }
 
