@@ -68,3 +68,25 @@ def test_traffic_figure_only_for_the_captured_kernel(tmp_path, monkeypatch):
     assert bench.load_traffic("missing") is None
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "fedcba9876543210")
     assert bench.load_traffic("k") is None
+
+
+def test_fp8mma_cache_only_in_attention_mode(monkeypatch, capsys):
+    """--cache fp8mma times the FP8 tensor-core attention alone; the stream
+    line carries it as fp8_mma_stream, so the stream mode rejects it before
+    touching a GPU."""
+    import pytest
+    monkeypatch.setattr("sys.argv", ["bench.py", "--cache", "fp8mma"])
+    with pytest.raises(SystemExit) as e:
+        bench.main()
+    assert e.value.code == 2
+    assert "fp8_mma_stream" in capsys.readouterr().err
+
+
+def test_stream_attention_launch_counts():
+    """Launches per attention call as the bench counts them: one for a bf16
+    cache, two for an E4M3 cache (the staging pass or the V-scale pass, then
+    the attention kernel)."""
+    st = bench.Stream.__new__(bench.Stream)
+    st.caches = [types.SimpleNamespace(dtype="bf16"), types.SimpleNamespace(dtype="fp8")]
+    assert st.attention_launches(0) == 1
+    assert st.attention_launches(1) == 2
