@@ -16,8 +16,14 @@ Metric: latent frames/s through the 30-layer attention stack; the attention
 kernel's achieved TFLOP/s against the measured dense-bf16 peak goes in
 "roofline".
 
+The line also carries the same stream over an E4M3 KV cache (fp8_stream:
+bf16 staging copy, then the bf16 kernel; fp8_mma_stream: the FP8 tensor-core
+attention), the recache kernel's TFLOP/s and the separate RoPE and append
+entry points' HBM figures.
+
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-       [--cache bf16|fp8]
+       [--cache bf16|fp8] [--layers L] [--separate] [--no-fp8-stream] [--no-cpu-baseline]
+       python bench.py --mode attention|recache|append|rope [--workload wan|chunk] [--cache ...]
 Under torchrun each rank runs an independent replica (no collective on the
 data path; "replicas only"); rank 0 prints one JSON line.
 """
