@@ -208,13 +208,13 @@ __global__ void __launch_bounds__(1024) rope_apply_kernel(const RopeApplyParams 
   const int rows = p.B * p.F * p.N;
   const int r0 = blockIdx.x * kRopeTokens;
   const int nt = min(kRopeTokens, rows - r0);
-  if (threadIdx.x < nt) {
-    const int tok = (r0 + threadIdx.x) % (p.F * p.N);
+  for (int k = threadIdx.x; k < nt; k += blockDim.x) {  // blockDim may be below kRopeTokens (H * D / 8 < 4)
+    const int tok = (r0 + k) % (p.F * p.N);
     const int fi = tok / p.N, n = tok - fi * p.N;
     const int r = n / p.rp.grid_w;
-    s_pos[threadIdx.x][0] = temporal_pos(p.rp, fi);
-    s_pos[threadIdx.x][1] = static_cast<float>(r);
-    s_pos[threadIdx.x][2] = static_cast<float>(n - r * p.rp.grid_w);
+    s_pos[k][0] = temporal_pos(p.rp, fi);
+    s_pos[k][1] = static_cast<float>(r);
+    s_pos[k][2] = static_cast<float>(n - r * p.rp.grid_w);
   }
   const int pth = p.rp.pt + p.rp.ph;
   float om[4];

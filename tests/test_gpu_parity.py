@@ -68,6 +68,18 @@ def test_rope_apply(name):
     assert_parity(np64(xg), ref, max_rel=tol, mean_abs=1e-3 if w.dtype != "f32" else 1e-6, what="rope")
 
 
+def test_rope_apply_one_head_d8():
+    """One head of D = 8 (a single 8-element chunk per token row, so a block
+    of the in-place RoPE has fewer threads than token rows), fp32, every
+    element checked."""
+    w = W.replace(W.TINY, H=1, D=8, pairs=(2, 1, 1), name="tiny_h1_d8")
+    x, _, _ = W.qkv_frames(w, 7, 5, 3)
+    xg = x.cuda()
+    swa.rope_apply(xg, 5, rope_of(w))
+    ref = orope.rope_frames(np64(x), 5, w.grid_h, w.grid_w, omega_of(w), w.pairs, w.t_offset)
+    assert_parity(np64(xg), ref, max_rel=1e-5, mean_abs=1e-6, what="rope h1 d8")
+
+
 @pytest.mark.parametrize("name", ["tiny", "chunk"])
 def test_rope_position_interpolation(name):
     """Position interpolation (t_scale): against the oracle at scale 1/4, and
