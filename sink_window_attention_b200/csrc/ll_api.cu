@@ -476,23 +476,20 @@ ll_status ll_kvcache_append(const ll_kvcache* cache, const void* k, const void* 
   p.first_frame = first_frame;
   if (slots_out)
     for (int i = 0; i < n_frames; ++i) ll_slot_of_frame(first_frame + i, cache->n_sink, cache->n_local, &slots_out[i]);
-  // threads: one per (token, 8-element chunk, group of append_heads_per_thread(H) heads)
-  const long long threads = static_cast<long long>(p.B) * n_frames * p.N * (p.D / 8) *
-                            (p.H / ll::append_heads_per_thread(p.H));
-  if (threads >= (1LL << 31)) return fail(LL_ERR_UNSUPPORTED, "tensor too large for one call (%lld threads)", threads);
-  const long long want = (threads + 255) / 256;
-  const int grid = static_cast<int>(want < 8LL * num_sms() ? want : 8LL * num_sms());
-  const size_t smem = ll::append_smem_bytes(n_frames, p.H, p.D, p.rp.pt);
-  if (smem > 48 * 1024)
-    return fail(LL_ERR_UNSUPPORTED, "frequency tables of %zu bytes exceed 48 KiB (n_frames x H x pairs_t too large)",
-                smem);
+  // one thread per (head, 8-element chunk) of a token row, kAppendTokens rows per block
+  const long long chunks = static_cast<long long>(p.B) * n_frames * p.N * p.H * (p.D / 8);
+  if (chunks >= (1LL << 31)) return fail(LL_ERR_UNSUPPORTED, "tensor too large for one call (%lld chunks)", chunks);
+  if (p.H * (p.D / 8) > 1024) return fail(LL_ERR_UNSUPPORTED, "H * D / 8 = %d exceeds 1024", p.H * (p.D / 8));
+  const long long rows = static_cast<long long>(p.B) * n_frames * p.N;
+  const int grid = static_cast<int>((rows + ll::kAppendTokens - 1) / ll::kAppendTokens);
+  const int threads = (p.H * (p.D / 8) + 31) / 32 * 32;  // whole warps (the E4M3 row max shuffles)
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cache->dtype == LL_BF16)
-    ll::append_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 256, smem, s>>>(p);
+    ll::append_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, threads, 0, s>>>(p);
   else if (cache->dtype == LL_F32)
-    ll::append_kernel<float, float><<<grid, 256, smem, s>>>(p);
+    ll::append_kernel<float, float><<<grid, threads, 0, s>>>(p);
   else
-    ll::append_kernel<__nv_bfloat16, uint8_t><<<grid, 256, smem, s>>>(p);
+    ll::append_kernel<__nv_bfloat16, uint8_t><<<grid, threads, 0, s>>>(p);
   return check_launch("append_kernel");
 }
 

@@ -496,9 +496,106 @@ __device__ __forceinline__ void append_blocks(const AppendParams& p, int blk, in
   }
 }
 
+// ll_kvcache_append: one thread per (head, 8-element chunk) of a token row
+// (blockDim = H * D/8) and kAppendTokens token rows per block, as in the
+// in-place RoPE: a thread's 4 frequencies are evaluated once; each row's
+// position and cache row once per block (shared memory); the K and V loads of
+// all rows are issued before any rotation. The angles are the same products
+// position x frequency as append_blocks forms (which the fused E4M3 staging
+// kernel uses), so the cache rows are the same bits. E4M3: the D/8 lanes of a
+// (token, head) row reduce its max|x| by shuffles; blockDim is rounded up to
+// whole warps and the lanes past H * D/8 only take part in the shuffles.
+constexpr int kAppendTokens = 2;
+
 template <typename Tin, typename C>
-__global__ void __launch_bounds__(256) append_kernel(const AppendParams p) {
-  append_blocks<Tin, C>(p, blockIdx.x, gridDim.x);
+__global__ void __launch_bounds__(1024) append_kernel(const AppendParams p) {
+  __shared__ float s_pos[kAppendTokens][3];      // temporal, row and column position
+  __shared__ long long s_dst[kAppendTokens];     // cache token row (batch entry, slot, token)
+  const int cpr = p.D / 8;
+  const bool live = static_cast<int>(threadIdx.x) < p.H * cpr;
+  const int h = live ? threadIdx.x / cpr : 0, c = threadIdx.x - (threadIdx.x / cpr) * cpr;
+  const int FN = p.F * p.N, rows = p.B * FN;
+  const int r0 = blockIdx.x * kAppendTokens;
+  const int nt = min(kAppendTokens, rows - r0);
+  for (int k = threadIdx.x; k < nt; k += blockDim.x) {
+    const int b = (r0 + k) / FN, tok = (r0 + k) - b * FN;
+    const int fi = tok / p.N, n = tok - fi * p.N;
+    const int gw = p.rp.grid_w > 0 ? p.rp.grid_w : 1;
+    const int r = n / gw;
+    s_pos[k][0] = temporal_pos(p.rp, fi);
+    s_pos[k][1] = static_cast<float>(r);
+    s_pos[k][2] = static_cast<float>(n - r * gw);
+    const int S = p.n_sink + p.n_local;
+    s_dst[k] = (static_cast<long long>(b) * S + cache_slot(p.first_frame + fi, p.n_sink, p.n_local)) * p.N + n;
+  }
+  float om[4];
+  if (p.rp.enabled) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) om[q] = omega_of(p.rp, h, c * 4 + q);
+  }
+  const Tin* kin = static_cast<const Tin*>(p.k_in) + (static_cast<size_t>(r0) * p.H + h) * p.D + c * 8;
+  const Tin* vin = static_cast<const Tin*>(p.v_in) + (static_cast<size_t>(r0) * p.H + h) * p.D + c * 8;
+  float kx[kAppendTokens][8], vx[kAppendTokens][8];
+#pragma unroll
+  for (int k = 0; k < kAppendTokens; ++k) {
+    if (live && k < nt) {
+      load_chunk8<Tin>(kin + static_cast<size_t>(k) * p.H * p.D, kx[k]);
+      load_chunk8<Tin>(vin + static_cast<size_t>(k) * p.H * p.D, vx[k]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) kx[k][e] = vx[k][e] = 0.f;
+    }
+  }
+  __syncthreads();
+  const int pth = p.rp.pt + p.rp.ph;
+#pragma unroll
+  for (int k = 0; k < kAppendTokens; ++k) {
+    if (k >= nt) break;  // uniform across the block
+    if (p.rp.enabled) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int j = c * 4 + q;
+        const float pos = j < p.rp.pt ? s_pos[k][0] : (j < pth ? s_pos[k][1] : s_pos[k][2]);
+        float sn, cs;
+        sincos_reduced(pos * om[q], sn, cs);
+        const float x0 = kx[k][2 * q], x1 = kx[k][2 * q + 1];
+        kx[k][2 * q] = x0 * cs - x1 * sn;
+        kx[k][2 * q + 1] = x0 * sn + x1 * cs;
+      }
+    }
+    const size_t dst = (static_cast<size_t>(s_dst[k]) * p.H + h) * p.D + c * 8;
+    if constexpr (sizeof(C) == 1) {
+      // per (token, head) row: scale = max|x| / 448 over the row's D values,
+      // held by the cpr consecutive lanes of this head
+      float ka = 0.f, va = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        ka = fmaxf(ka, fabsf(kx[k][e]));
+        va = fmaxf(va, fabsf(vx[k][e]));
+      }
+      for (int off = cpr >> 1; off > 0; off >>= 1) {
+        ka = fmaxf(ka, __shfl_xor_sync(0xffffffffu, ka, off));
+        va = fmaxf(va, __shfl_xor_sync(0xffffffffu, va, off));
+      }
+      const float ks = ka > 0.f ? __fdiv_rn(ka, 448.0f) : 1.0f;
+      const float vs = va > 0.f ? __fdiv_rn(va, 448.0f) : 1.0f;
+      if (!live) continue;
+      const uint2 kq = encode_chunk8_e4m3(kx[k], ks), vq = encode_chunk8_e4m3(vx[k], vs);
+      *reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.k_cache) + dst) = kq;
+      *reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.v_cache) + dst) = vq;
+      if (p.stage_k != nullptr) {
+        *reinterpret_cast<uint4*>(p.stage_k + dst) = decode_chunk8_e4m3_bf16(kq, ks);
+        *reinterpret_cast<uint4*>(p.stage_v + dst) = decode_chunk8_e4m3_bf16(vq, vs);
+      }
+      if (c == 0) {
+        p.k_scale[dst / p.D] = ks;
+        p.v_scale[dst / p.D] = vs;
+      }
+    } else if (live) {
+      store_chunk8<C>(static_cast<C*>(p.k_cache) + dst, kx[k]);
+      store_chunk8<C>(static_cast<C*>(p.v_cache) + dst, vx[k]);
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
