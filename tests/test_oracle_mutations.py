@@ -17,9 +17,11 @@ What each mistake contradicts:
 - 3 sink frames + 9 local frames including the current one (LongLive review,
   'Short-Window Attention', 'Frame Sink');
 - RMSNorm over the row (y = x / sqrt(mean x^2 + eps) * gamma) and RoPE at the
-  frame's own position ('KV Recache');
+  frame's own position ('KV Recache'), on K = X Wk only, V = X Wv stored as
+  is (the reading the oracle states for the recompute);
 - the OCP E4M3 encoding (bias 7, subnormals without the implicit one,
-  round to nearest even, 448 as the largest finite value).
+  round to nearest even, 448 as the largest finite value) and the per-row
+  scale that multiplies the decoded codes back.
 """
 import json
 import os
@@ -390,6 +392,47 @@ def quantize_to_240(x):
     return fp8.e4m3_encode(x / scale[..., None]), scale
 
 
+def _recache_parts(x, wk, wv):
+    x = np.asarray(x, dtype=np.float64)
+    return x @ np.asarray(wk, dtype=np.float64), x @ np.asarray(wv, dtype=np.float64)
+
+
+def recache_wk_wv_swapped(x, wk, wv, gamma, eps, frame, H, D, grid_h, grid_w, omega, pairs,
+                          t_offset=0, t_scale=1.0):
+    return recache.__dict__["_recache_orig"](x, wv, wk, gamma, eps, frame, H, D, grid_h, grid_w, omega, pairs,
+                                             t_offset, t_scale)
+
+
+def recache_v_rotated_too(x, wk, wv, gamma, eps, frame, H, D, grid_h, grid_w, omega, pairs,
+                          t_offset=0, t_scale=1.0):
+    k, v = recache.__dict__["_recache_orig"](x, wk, wv, gamma, eps, frame, H, D, grid_h, grid_w, omega, pairs,
+                                             t_offset, t_scale)
+    t, r, c = rope.token_positions(frame, grid_h, grid_w, t_offset, t_scale)
+    return k, rope.rope_3d(v, t, r, c, omega, pairs)
+
+
+def recache_k_not_normalised(x, wk, wv, gamma, eps, frame, H, D, grid_h, grid_w, omega, pairs,
+                             t_offset=0, t_scale=1.0):
+    kp, vp = _recache_parts(x, wk, wv)
+    t, r, c = rope.token_positions(frame, grid_h, grid_w, t_offset, t_scale)
+    k = (kp * np.asarray(gamma, dtype=np.float64)).reshape(-1, H, D)
+    return rope.rope_3d(k, t, r, c, omega, pairs), vp.reshape(-1, H, D)
+
+
+def recache_rotated_one_frame_late(x, wk, wv, gamma, eps, frame, H, D, grid_h, grid_w, omega, pairs,
+                                   t_offset=0, t_scale=1.0):
+    return recache.__dict__["_recache_orig"](x, wk, wv, gamma, eps, frame + 1, H, D, grid_h, grid_w, omega,
+                                             pairs, t_offset, t_scale)
+
+
+def dequantize_dividing(codes, scale):
+    return fp8.e4m3_decode_array(codes) / np.asarray(scale, dtype=np.float64)[..., None]
+
+
+def dequantize_without_sign(codes, scale):
+    return np.abs(fp8.e4m3_decode_array(codes)) * np.asarray(scale, dtype=np.float64)[..., None]
+
+
 RECACHE_CASES = {
     "RMS over the tokens instead of the row": (recache, "rmsnorm", rms_over_tokens, [pin_rf.test_rmsnorm_textbook]),
     "eps outside the square root": (recache, "rmsnorm", rms_eps_outside_root, [pin_rf.test_rmsnorm_textbook]),
@@ -404,6 +447,18 @@ RECACHE_CASES = {
     "E4M3 encode truncating": (fp8, "_encode_magnitudes", encode_truncating,
                                [lambda: pin_rf.test_e4m3_golden(golden), pin_rf.test_e4m3_encode_roundtrip_and_nearest]),
     "E4M3 row scale for 240 instead of 448": (fp8, "quantize_rows", quantize_to_240, [pin_rf.test_quantize_rows]),
+    "recache with Wk and Wv swapped": (recache, "recache_frame", recache_wk_wv_swapped,
+                                       [pin_rf.test_recache_frame_composition]),
+    "recache rotating V as well": (recache, "recache_frame", recache_v_rotated_too,
+                                   [pin_rf.test_recache_frame_composition]),
+    "recache K without the RMSNorm": (recache, "recache_frame", recache_k_not_normalised,
+                                      [pin_rf.test_recache_frame_composition]),
+    "recache RoPE one frame late": (recache, "recache_frame", recache_rotated_one_frame_late,
+                                    [pin_rf.test_recache_frame_composition]),
+    "E4M3 dequantise dividing by the scale": (fp8, "dequantize_rows", dequantize_dividing,
+                                              [pin_rf.test_quantize_rows]),
+    "E4M3 dequantise dropping the sign": (fp8, "dequantize_rows", dequantize_without_sign,
+                                          [pin_rf.test_quantize_rows]),
 }
 
 
