@@ -14,8 +14,9 @@ What each mistake contradicts:
 - the row-major (h, w) token order and the t, h, w band order of the 3D RoPE;
 - C(Delta) = (1/K) sum_i e^{j w_i Delta} ('Core innovation');
 - softmax(Q K^T / sqrt(d)) V ('Multi-head attention');
-- 3 sink frames + 9 local frames including the current one (LongLive review,
-  'Short-Window Attention', 'Frame Sink');
+- 3 sink frames + 9 local frames including the current one, the sinks pinned
+  and the local frames in a ring (LongLive review, 'Short-Window Attention',
+  'Frame Sink'; LoL review, 'Attention Sink');
 - RMSNorm over the row (y = x / sqrt(mean x^2 + eps) * gamma) and RoPE at the
   frame's own position ('KV Recache'), on K = X Wk only, V = X Wv stored as
   is (the reading the oracle states for the recompute);
@@ -302,6 +303,35 @@ def test_window_attention_pin_rejects_missing_sinks(monkeypatch):
     assert rejected(pin)
 
 
+def probabilities_scale_one_over_d(q, k, scale=None):
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    return attention.softmax_rows(np.einsum("qhd,khd->hqk", q, k) / q.shape[-1])
+
+
+def frame_causal_one_frame_short(q_rot_frames, k_rot_frames, v_frames, query_frame, N, scale=None):
+    q = q_rot_frames[query_frame * N:(query_frame + 1) * N]
+    hi = max(query_frame, 1) * N
+    return attention.mha(q, k_rot_frames[:hi], v_frames[:hi], scale)
+
+
+def test_probability_pin_rejects_wrong_scale(monkeypatch):
+    """attention_probabilities is held to the hand-worked example."""
+    pin = [lambda: pin_att.test_worked_example(golden)]
+    assert not rejected(pin)
+    monkeypatch.setattr(attention, "attention_probabilities", probabilities_scale_one_over_d)
+    assert rejected(pin)
+
+
+def test_full_window_pin_rejects_a_short_frame_causal_reference(monkeypatch):
+    """With a window longer than the stream the stream oracle must equal full
+    frame-causal attention over frames 0..f, the current frame included."""
+    pin = [lambda: pin_att.test_stream_matches_dense_masked_brute_force(10_000, 1)]
+    assert not rejected(pin)
+    monkeypatch.setattr(attention, "frame_causal_attention", frame_causal_one_frame_short)
+    assert rejected(pin)
+
+
 # ------------------------------------------------------------------ window and slots
 def attended_local_one_short(f, n_sink=3, n_local=9):
     if f < 0:
@@ -319,6 +349,29 @@ def slot_ring_off_by_one(f, n_sink=3, n_local=9):
     return f if f < n_sink else n_sink + (f - n_sink + 1) % n_local
 
 
+def slot_ring_over_every_slot(f, n_sink=3, n_local=9):
+    if f < 0:
+        raise ValueError("negative frame index")
+    return f % (n_sink + n_local)
+
+
+def valid_slots_one_short(f, n_sink=3, n_local=9):
+    return min(f, n_sink + n_local)
+
+
+def valid_slots_capped_at_local(f, n_sink=3, n_local=9):
+    return min(f + 1, n_local)
+
+
+def slot_frames_first_writer_kept(last_frame, n_sink=3, n_local=9):
+    held = [-1] * (n_sink + n_local)
+    for g in range(last_frame + 1):
+        s = window.slot_of(g, n_sink, n_local)
+        if held[s] < 0:
+            held[s] = g
+    return held
+
+
 WINDOW_PINS = [lambda: pin_win.test_attended_golden(golden),
                lambda: pin_win.test_slot_map_matches_brute_force(3, 9, 1),
                lambda: pin_win.test_slot_map_matches_brute_force(3, 9, 3)]
@@ -326,6 +379,10 @@ WINDOW_CASES = {
     "local window one frame short": ("attended_frames", attended_local_one_short),
     "no sink frames (last 12 frames)": ("attended_frames", attended_without_sinks),
     "ring slot off by one": ("slot_of", slot_ring_off_by_one),
+    "ring over every slot (sinks evicted)": ("slot_of", slot_ring_over_every_slot),
+    "valid slot count one short": ("valid_slots", valid_slots_one_short),
+    "valid slot count capped at the local window": ("valid_slots", valid_slots_capped_at_local),
+    "slot map keeping the first frame written": ("slot_frames", slot_frames_first_writer_kept),
 }
 
 
