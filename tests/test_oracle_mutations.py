@@ -132,6 +132,19 @@ def coherence_without_mean(omega, deltas):
     return np.exp(1j * omega[None, :] * deltas[:, None]).sum(axis=1)
 
 
+def positions_without_t_offset(frame, grid_h, grid_w, t_offset=0, t_scale=1.0):
+    return rope.__dict__["_positions_orig"](frame, grid_h, grid_w, 0, t_scale)
+
+
+def positions_offset_not_interpolated(frame, grid_h, grid_w, t_offset=0, t_scale=1.0):
+    t, r, c = rope.__dict__["_positions_orig"](frame, grid_h, grid_w, 0, t_scale)
+    return t + t_offset, r, c
+
+
+def rope_frames_from_frame_zero(x, first_frame, grid_h, grid_w, omega, pairs, t_offset=0, t_scale=1.0):
+    return rope.__dict__["_rope_frames_orig"](x, 0, grid_h, grid_w, omega, pairs, t_offset, t_scale)
+
+
 ROPE_CASES = {
     "rotation sign flipped": ("rotate_pairs", rot_sign_flipped,
                               [lambda: pin_rope.test_rotation_golden(golden),
@@ -162,10 +175,22 @@ ROPE_CASES = {
 }
 
 
+ROPE_CASES.update({
+    "t offset dropped": ("token_positions", positions_without_t_offset,
+                         [pin_rope.test_token_positions_row_major, pin_rope.test_rope_frames_absolute_positions]),
+    "interpolation not applied to the t offset": ("token_positions", positions_offset_not_interpolated,
+                                                  [pin_rope.test_rope_frames_absolute_positions]),
+    "a block of frames rotated from frame 0": ("rope_frames", rope_frames_from_frame_zero,
+                                               [pin_rope.test_rope_frames_absolute_positions]),
+})
+
+
 @pytest.mark.parametrize("case", sorted(ROPE_CASES))
 def test_rope_pins_reject(case, monkeypatch):
     name, wrong, pins = ROPE_CASES[case]
     assert not rejected(pins), "the pins must pass on the oracle as written"
+    monkeypatch.setitem(rope.__dict__, "_positions_orig", rope.token_positions)
+    monkeypatch.setitem(rope.__dict__, "_rope_frames_orig", rope.rope_frames)
     monkeypatch.setattr(rope, name, wrong)
     assert rejected(pins), case
 

@@ -143,6 +143,30 @@ def test_token_positions_row_major():
     assert r[-1] == 3 and c[-1] == 5
 
 
+def test_rope_frames_absolute_positions():
+    """Every token of a block of frames turns by its own absolute position: the
+    first pair of each band has frequency 1 (i = 0), so in frame g of the block
+    its t pair turns by exactly (t_offset + g) * t_scale radians and its h and w
+    pairs by the token's row and column, written out with math.cos / math.sin."""
+    pairs = (12, 10, 10)
+    H, gh, gw = 2, 2, 3
+    N = gh * gw
+    om = rope.head_frequencies(H, pairs, 10000.0)
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((2, 3 * N, H, 64))
+    first, t_offset, t_scale = 5, 100, 0.5
+    y = rope.rope_frames(x, first, gh, gw, om, pairs, t_offset, t_scale)
+    for b in range(2):
+        for fi in range(3):
+            for n in range(N):
+                row = fi * N + n
+                for j, ang in [(0, (t_offset + first + fi) * t_scale), (2 * 12, n // gw), (2 * 22, n % gw)]:
+                    x0, x1 = x[b, row, :, j], x[b, row, :, j + 1]
+                    c, s_ = math.cos(ang), math.sin(ang)
+                    assert np.allclose(y[b, row, :, j], c * x0 - s_ * x1, atol=1e-12)
+                    assert np.allclose(y[b, row, :, j + 1], s_ * x0 + c * x1, atol=1e-12)
+
+
 # ---------------------------------------------------------------- phase coherence and position interpolation
 def test_phase_coherence_special_values():
     """C(0) = 1, |C| <= 1, C(-D) = conj C(D); one component is a pure phase."""
