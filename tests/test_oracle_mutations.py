@@ -302,6 +302,41 @@ def test_stream_pins_reject_lost_denoising_pass_and_lost_interpolation(monkeypat
         assert rejected(pi)
 
 
+def attend_window_of_the_first_frame(self, q, first_frame, scale=None, rows=None, return_lse=False):
+    qr = self.rotate_queries(q, first_frame)
+    if rows is not None:
+        qr = qr[np.asarray(rows)]
+    return attention.sink_window_attention(qr, self.k, self.v, first_frame, self.n_sink, self.n_local, scale,
+                                           return_lse)
+
+
+def queries_not_rotated(self, q, first_frame):
+    return np.asarray(q, dtype=np.float64)
+
+
+def queries_all_at_the_first_frame(self, q, first_frame):
+    q = np.asarray(q, dtype=np.float64)
+    F = q.shape[0] // self.N
+    return np.concatenate([self._rot(q[fi * self.N:(fi + 1) * self.N], first_frame) for fi in range(F)], axis=0)
+
+
+STREAM_PINS = [lambda: pin_att.test_stream_matches_dense_masked_brute_force(9, 1),
+               lambda: pin_att.test_stream_matches_dense_masked_brute_force(9, 3)]
+STREAM_CASES = {
+    "a chunk attending with its first frame's window": ("attend", attend_window_of_the_first_frame),
+    "queries not rotated": ("rotate_queries", queries_not_rotated),
+    "every query frame of a chunk rotated at the first": ("rotate_queries", queries_all_at_the_first_frame),
+}
+
+
+@pytest.mark.parametrize("case", sorted(STREAM_CASES))
+def test_stream_pins_reject(case, monkeypatch):
+    name, wrong = STREAM_CASES[case]
+    assert not rejected(STREAM_PINS)
+    monkeypatch.setattr(StreamOracle, name, wrong)
+    assert rejected(STREAM_PINS), case
+
+
 def test_stream_pin_rejects_keys_rotated_at_their_slot(monkeypatch):
     """K must turn with its frame's absolute position, not its cache slot."""
     pin = [lambda: pin_att.test_stream_matches_dense_masked_brute_force(9, 1)]
