@@ -602,10 +602,12 @@ STEP_TARGET_S = 3.0
 
 
 def oracle_rows(ora: "OracleStep") -> int:
-    """Query rows per sample: a 64-row probe (the faster of two, the first
-    pays for page faults) scaled to STEP_TARGET_S."""
-    t64 = min(ora.time(64), ora.time(64))
-    return int(max(64, min(ora.w.N, 64 * STEP_TARGET_S / max(t64, 1e-3))))
+    """Query rows per sample: a probe of 64 rows (all of them in a frame of
+    fewer; the faster of two runs, the first pays for page faults) scaled to
+    STEP_TARGET_S, never fewer rows than the probe nor more than a frame."""
+    probe = min(64, ora.w.N)
+    t = min(ora.time(probe), ora.time(probe))
+    return int(max(probe, min(ora.w.N, probe * STEP_TARGET_S / max(t, 1e-3))))
 
 
 def oracle_sample_desc(w: W.Workload, rows: int) -> str:

@@ -1,7 +1,8 @@
 """Host logic of bench.py that needs no GPU: the algorithmic FLOP and byte
 counts behind the roofline, the clock-sample parsing that decides whether a
 run is kept, the frames a recache recomputes, and the DRAM figure taken from
-a committed ncu summary."""
+a committed ncu summary, and what the reference arm (the oracle on the host
+cores) reports."""
 import types
 
 import bench
@@ -90,3 +91,39 @@ def test_stream_attention_launch_counts():
     st.caches = [types.SimpleNamespace(dtype="bf16"), types.SimpleNamespace(dtype="fp8")]
     assert st.attention_launches(0) == 1
     assert st.attention_launches(1) == 2
+
+
+def test_reference_arm_reports_what_it_timed(monkeypatch):
+    """The reference arm (the oracle on the host cores) on a small stream:
+    rank 0 alone prints; ms_per_step is the mean of the timed samples, value
+    is the latent frames those samples amount to per second, and the
+    whole-frame figure is kept apart as an extrapolation."""
+    small = W.replace(W.STREAM, grid_h=4, grid_w=6, H=2, D=64, pairs=(12, 10, 10), layers=3)
+    monkeypatch.setattr(bench.W, "STREAM", small)
+    monkeypatch.setattr(bench, "STEP_TARGET_S", 0.01)
+    timed = []
+    orig = bench.OracleStep.time
+
+    def record(self, rows):
+        t = orig(self, rows)
+        timed.append((rows, t))
+        return t
+
+    monkeypatch.setattr(bench.OracleStep, "time", record)
+    args = types.SimpleNamespace(steps=3, warmup=2)
+    assert bench.run_reference(args, 1, 2) is None
+    assert timed == []
+    line = bench.run_reference(args, 0, 1)
+    rows = timed[-1][0]
+    assert rows == small.N == 24                         # a frame of fewer than 64 rows: all of them
+    samples = [t for _, t in timed[-3:]]
+    assert len(timed) == 2 + 2 + 3                       # two probes, warm-up, timed steps
+    assert abs(line["ms_per_step"] - sum(samples) / 3 * 1e3) <= 1e-3
+    frames = rows / small.N / small.layers
+    assert abs(line["value"] - frames / (sum(samples) / 3)) <= 1e-6 * max(1.0, line["value"])
+    assert line["impl"] == "reference" and line["higher_is_better"] is True and line["dtype"] == "f64"
+    assert line["steps"] == 3 and line["warmup"] == 2 and line["n_gpus"] == 1
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    assert "not a measurement" in line["extrapolated"]["note"]
