@@ -132,6 +132,30 @@ def coherence_without_mean(omega, deltas):
     return np.exp(1j * omega[None, :] * deltas[:, None]).sum(axis=1)
 
 
+def jitter_of_head_zero_for_all(H, pairs, theta0, sigma=0.0, eps=None):
+    if eps is not None:
+        eps = np.full(H, np.asarray(eps, dtype=np.float64)[0])
+    return rope.__dict__["_head_freq_orig"](H, pairs, theta0, sigma, eps)
+
+
+def jitter_added_not_scaled(theta0, sigma, eps):
+    return theta0 + sigma * np.asarray(eps, dtype=np.float64)
+
+
+def rot_half_angle(x, angle):
+    return rope.__dict__["_rotate_orig"](x, 0.5 * np.asarray(angle, dtype=np.float64))
+
+
+def spatial_bands_with_temporal_width(H, pairs, theta0, sigma=0.0, eps=None):
+    pt, ph, pw = pairs
+    out = rope.__dict__["_head_freq_orig"](H, pairs, theta0, sigma, eps)
+    i_h = np.arange(ph, dtype=np.float64)
+    i_w = np.arange(pw, dtype=np.float64)
+    out[:, pt:pt + ph] = np.power(float(theta0), -2.0 * i_h / (2 * pt))
+    out[:, pt + ph:] = np.power(float(theta0), -2.0 * i_w / (2 * pt))
+    return out
+
+
 def positions_without_t_offset(frame, grid_h, grid_w, t_offset=0, t_scale=1.0):
     return rope.__dict__["_positions_orig"](frame, grid_h, grid_w, 0, t_scale)
 
@@ -182,6 +206,14 @@ ROPE_CASES.update({
                                                   [pin_rope.test_rope_frames_absolute_positions]),
     "a block of frames rotated from frame 0": ("rope_frames", rope_frames_from_frame_zero,
                                                [pin_rope.test_rope_frames_absolute_positions]),
+    "every head given head 0's jitter": ("head_frequencies", jitter_of_head_zero_for_all,
+                                         [pin_rope.test_jitter_regenerated_from_seed]),
+    "jitter added to theta0 instead of scaling it": ("jittered_base", jitter_added_not_scaled,
+                                                     [lambda: pin_rope.test_jitter_points_and_bounds(golden)]),
+    "rotation by half the angle": ("rotate_pairs", rot_half_angle,
+                                   [lambda: pin_rope.test_rotation_golden(golden)]),
+    "spatial bands with the temporal band's width": ("head_frequencies", spatial_bands_with_temporal_width,
+                                                      [pin_rope.test_jitter_regenerated_from_seed]),
 })
 
 
@@ -191,6 +223,8 @@ def test_rope_pins_reject(case, monkeypatch):
     assert not rejected(pins), "the pins must pass on the oracle as written"
     monkeypatch.setitem(rope.__dict__, "_positions_orig", rope.token_positions)
     monkeypatch.setitem(rope.__dict__, "_rope_frames_orig", rope.rope_frames)
+    monkeypatch.setitem(rope.__dict__, "_head_freq_orig", rope.head_frequencies)
+    monkeypatch.setitem(rope.__dict__, "_rotate_orig", rope.rotate_pairs)
     monkeypatch.setattr(rope, name, wrong)
     assert rejected(pins), case
 
