@@ -156,6 +156,18 @@ def spatial_bands_with_temporal_width(H, pairs, theta0, sigma=0.0, eps=None):
     return out
 
 
+def coherence_real_part_only(omega, deltas):
+    omega = np.asarray(omega, dtype=np.float64)
+    deltas = np.asarray(deltas, dtype=np.float64)
+    return np.cos(omega[None, :] * deltas[:, None]).mean(axis=1).astype(np.complex128)
+
+
+def coherence_conjugate_phase(omega, deltas):
+    omega = np.asarray(omega, dtype=np.float64)
+    deltas = np.asarray(deltas, dtype=np.float64)
+    return np.exp(-1j * omega[None, :] * deltas[:, None]).mean(axis=1)
+
+
 def positions_without_t_offset(frame, grid_h, grid_w, t_offset=0, t_scale=1.0):
     return rope.__dict__["_positions_orig"](frame, grid_h, grid_w, 0, t_scale)
 
@@ -206,6 +218,12 @@ ROPE_CASES.update({
                                                   [pin_rope.test_rope_frames_absolute_positions]),
     "a block of frames rotated from frame 0": ("rope_frames", rope_frames_from_frame_zero,
                                                [pin_rope.test_rope_frames_absolute_positions]),
+    "coherence from the real parts only": ("phase_coherence", coherence_real_part_only,
+                                           [pin_rope.test_phase_coherence_special_values,
+                                            pin_rope.test_phase_coherence_harmonic_closed_form]),
+    "coherence with the conjugate phase": ("phase_coherence", coherence_conjugate_phase,
+                                           [pin_rope.test_phase_coherence_special_values,
+                                            pin_rope.test_phase_coherence_harmonic_closed_form]),
     "every head given head 0's jitter": ("head_frequencies", jitter_of_head_zero_for_all,
                                          [pin_rope.test_jitter_regenerated_from_seed]),
     "jitter added to theta0 instead of scaling it": ("jittered_base", jitter_added_not_scaled,
