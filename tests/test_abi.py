@@ -1,6 +1,8 @@
 """The C ABI without a GPU: the library loads, exports every function that
-include/ll_api.h declares, maps frames to slots bit-exactly, and rejects bad
-arguments on the host before anything is launched."""
+include/ll_api.h declares, the binding passes each argument with the
+header's type and lays out its structures as the C compiler does, frames map
+to slots bit-exactly, and bad arguments are rejected on the host before
+anything is launched."""
 import ctypes
 import os
 import re
@@ -298,3 +300,81 @@ def test_workspace_sizes_and_noalloc_limit(L):
     staging = 2 * align(12 * 1560 * 12 * 128 * 2)
     assert ws(fp8, 1) == ws(_cache(), 1) + staging
     assert ws(_cache(), 0) == 0 and L.ll_sink_window_attention_workspace_bytes(None, 1) == 0
+
+
+def _prototypes():
+    """(return type, name, [parameter types]) of every function in ll_api.h."""
+    src = open(os.path.join(ROOT, "include", "ll_api.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    out = []
+    for m in re.finditer(r"([A-Za-z_][A-Za-z0-9_ \*]*?)\b(ll_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", src, flags=re.S):
+        params = [p.strip() for p in m.group(3).split(",")]
+        if params == ["void"]:
+            params = []
+        # drop the parameter name, keep its type
+        types_ = [re.sub(r"\s*\b[A-Za-z_][A-Za-z0-9_]*$", "", p) if not p.endswith("*") else p for p in params]
+        out.append((m.group(1).strip(), m.group(2), [" ".join(t.replace("*", " * ").split()) for t in types_]))
+    return out
+
+
+def _ctype_of(c_type: str):
+    """The ctypes type the binding must pass for a C parameter type."""
+    t = c_type.replace("const ", "").strip()
+    if t == "ll_rope_desc *":
+        return ctypes.POINTER(swa.RopeDescC)
+    if t == "ll_kvcache *":
+        return ctypes.POINTER(swa.KVCacheC)
+    if t == "long long *":
+        return ctypes.POINTER(ctypes.c_longlong)
+    if t == "int *":
+        return ctypes.POINTER(ctypes.c_int)
+    if t.endswith("*"):
+        return ctypes.c_void_p                      # device or host buffers, streams
+    return {"int": ctypes.c_int, "ll_dtype": ctypes.c_int, "ll_status": ctypes.c_int, "long long": ctypes.c_longlong,
+            "float": ctypes.c_float, "double": ctypes.c_double, "size_t": ctypes.c_size_t}[t]
+
+
+def test_binding_signatures_match_the_header(L):
+    """Every argtypes / restype the binding sets agrees with the prototype in
+    ll_api.h, parameter by parameter (count, integer widths, float vs double,
+    pointers), so the marshalling cannot shift or truncate an argument."""
+    protos = _prototypes()
+    assert sorted(n for _, n, _ in protos) == sorted(swa.EXPORTED)
+    for ret, name, params in protos:
+        fn = getattr(L, name)
+        want = [_ctype_of(p) for p in params]
+        got = fn.argtypes
+        if want:
+            assert got is not None and len(got) == len(want), (name, got, params)
+            for g, w, p in zip(got, want, params):
+                if w is ctypes.c_void_p:
+                    assert g is ctypes.c_void_p or issubclass(g, ctypes._Pointer), (name, p, g)
+                else:
+                    assert g is w, (name, p, g, w)
+        rt = ctypes.c_char_p if ret == "const char*" else _ctype_of(ret)
+        assert fn.restype is rt, (name, ret, fn.restype)
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """sizeof and offsetof of every field of ll_rope_desc and ll_kvcache, as
+    gcc lays out the header, equal the ctypes structures of the binding."""
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "ll_api.h"', "int main(void) {"]
+    for cname, cls in (("ll_rope_desc", swa.RopeDescC), ("ll_kvcache", swa.KVCacheC)):
+        lines.append(f'  printf("{cname} sizeof %zu\\n", sizeof({cname}));')
+        for field, _ in cls._fields_:
+            lines.append(f'  printf("{cname} {field} %zu\\n", offsetof({cname}, {field}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    import subprocess
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.splitlines():
+        s, f, v = line.split()
+        got[(s, f)] = int(v)
+    for cname, cls in (("ll_rope_desc", swa.RopeDescC), ("ll_kvcache", swa.KVCacheC)):
+        assert got[(cname, "sizeof")] == ctypes.sizeof(cls), cname
+        for field, _ in cls._fields_:
+            assert got[(cname, field)] == getattr(cls, field).offset, (cname, field)
