@@ -378,3 +378,39 @@ def test_struct_layouts_match_the_header(tmp_path):
         assert got[(cname, "sizeof")] == ctypes.sizeof(cls), cname
         for field, _ in cls._fields_:
             assert got[(cname, field)] == getattr(cls, field).offset, (cname, field)
+
+
+def test_plain_c_program_links_and_calls_the_library(L, tmp_path):
+    """The boundary is usable from C alone: a program built by gcc against
+    ll_api.h and linked with libll_swa.so (no Python, no PyTorch) reads the ABI
+    version, maps frames to slots and gets a host-side rejection with its
+    message, none of which needs a GPU."""
+    import subprocess
+    lib_dir = os.path.dirname(swa.LIB_PATH)
+    src = tmp_path / "use_abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "ll_api.h"
+int main(void) {
+  if (ll_abi_version() != LL_ABI_VERSION) return 1;
+  int slot = -1;
+  if (ll_slot_of_frame(100, 3, 9, &slot) != LL_OK || slot != 3 + (100 - 3) % 9) return 2;
+  if (ll_slot_of_frame(2, 3, 9, &slot) != LL_OK || slot != 2) return 3;
+  ll_rope_desc rope;
+  memset(&rope, 0, sizeof(rope));
+  rope.pairs_t = 10; rope.pairs_h = 10; rope.pairs_w = 10;   /* sums to 30, not D/2 = 32 */
+  rope.theta0 = 10000.0; rope.grid_h = 2; rope.grid_w = 3;
+  if (ll_rope_apply((void*)0, LL_BF16, 1, 1, 2, 64, 0, &rope, (void*)0) != LL_ERR_INVALID_ARG) return 4;
+  const char* msg = ll_last_error();
+  if (msg == NULL || strlen(msg) == 0) return 5;
+  printf("%s\n", msg);
+  return 0;
+}
+''')
+    exe = tmp_path / "use_abi"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                    "-L", lib_dir, "-l:" + os.path.basename(swa.LIB_PATH), "-Wl,-rpath," + lib_dir], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
+    assert r.stdout.strip()
