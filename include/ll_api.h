@@ -340,7 +340,9 @@ ll_status ll_sink_window_attention_noalloc(const void* q, ll_dtype q_dtype, cons
  * slot_frames: HOST array of n_slots absolute frame indices (frame in slot s),
  * each in [0, 2^31 - 1].
  * workspace: device scratch of at least ll_kv_recache_workspace_bytes(...)
- * bytes. The cache may be BF16 or FP8.
+ * bytes (0 in this build, where the row sums of the RMSNorm are exchanged on
+ * chip between the CTAs of a cluster; NULL is then allowed). The cache may be
+ * BF16 or FP8.
  * Errors: LL_ERR_INVALID_ARG for NULL or misaligned pointers, n_slots outside
  * [1, S], frames outside [0, 2^31 - 1]; LL_ERR_UNSUPPORTED for a d_model that
  * is not a positive multiple of 64, for H*D that is not a multiple of 256 up
