@@ -127,3 +127,27 @@ def test_reference_arm_reports_what_it_timed(monkeypatch):
     assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
     assert "not a measurement" in line["extrapolated"]["note"]
+
+
+def test_cpu_baseline_repeats_the_sample_to_its_time_budget(monkeypatch):
+    """Our arm's cpu_baseline repeats the oracle sample until the budget is
+    spent and reports the frames of all samples over their summed time."""
+    small = W.replace(W.STREAM, grid_h=4, grid_w=6, H=2, D=64, pairs=(12, 10, 10), layers=3)
+    monkeypatch.setattr(bench, "STEP_TARGET_S", 0.01)
+    monkeypatch.setattr(bench, "BASELINE_TARGET_S", 0.05)
+    timed = []
+    orig = bench.OracleStep.time
+
+    def record(self, rows):
+        t = orig(self, rows)
+        timed.append(t)
+        return t
+
+    monkeypatch.setattr(bench.OracleStep, "time", record)
+    cb = bench.cpu_baseline(small)
+    samples = timed[2:]                                   # after the two probes
+    assert 1 <= len(samples) <= bench.BASELINE_MAX_SAMPLES
+    assert sum(samples) >= 0.05 or len(samples) == bench.BASELINE_MAX_SAMPLES
+    frames = len(samples) * small.N / small.N / small.layers
+    assert abs(cb["value"] - frames / sum(samples)) <= 1e-6 + 1e-6 * cb["value"]
+    assert cb["kind"] == "oracle" and cb["sample"].startswith(f"{len(samples)} consecutive samples")
