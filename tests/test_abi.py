@@ -414,3 +414,14 @@ int main(void) {
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
     assert r.stdout.strip()
+
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=400, deadline=None)
+@given(frame=st.integers(0, 2**62), n_sink=st.integers(0, 64), n_local=st.integers(1, 64))
+def test_slot_map_bit_exact_random(L, frame, n_sink, n_local):
+    """The library's slot map (a host helper; the kernels compute the same
+    map on the device) equals the oracle's for any frame index and window."""
+    assert swa.slot_of_frame(frame, n_sink, n_local) == window.slot_of(frame, n_sink, n_local)

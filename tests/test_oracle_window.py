@@ -62,3 +62,21 @@ def test_window_covers_everything_when_large():
     # with a window at least as long as the stream, A(f) = 0..f (full frame-causal)
     for f in range(50):
         assert window.attended_frames(f, 3, 1000) == list(range(f + 1))
+
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=150, deadline=None)
+@given(n_sink=st.integers(0, 6), n_local=st.integers(1, 14), chunk=st.integers(1, 4), n_frames=st.integers(1, 80))
+def test_slot_map_matches_brute_force_random(n_sink, n_local, chunk, n_frames):
+    """The brute-force cache simulation above, over random windows, chunk
+    sizes (up to the local window) and stream lengths."""
+    if chunk > n_local:
+        chunk = n_local
+    for g, s, slots in _simulate(n_frames, n_sink, n_local, chunk):
+        assert window.slot_of(g, n_sink, n_local) == s
+        held = [x for x in slots if x is not None]
+        assert sorted(held) == window.attended_frames(g, n_sink, n_local)
+        nv = window.valid_slots(g, n_sink, n_local)
+        assert all(x is not None for x in slots[:nv]) and all(x is None for x in slots[nv:])
