@@ -61,6 +61,12 @@ def attention_flops(w: W.Workload) -> float:
     return 4.0 * nq * nk * w.D * w.H
 
 
+def recache_flops(w: W.Workload) -> float:
+    """Algorithmic FLOPs of one layer's recache: X [S*N, d_model] times
+    [Wk | Wv] [d_model, 2*H*D] (the RMSNorm and RoPE epilogue not counted)."""
+    return 2.0 * (w.slots * w.N) * w.dm * (2 * w.H * w.D)
+
+
 def append_bytes(w: W.Workload, cache_elem: int) -> float:
     """Algorithmic HBM bytes of one append: read K, V (bf16) and write them to the cache."""
     n = w.N * w.H * w.D
@@ -353,7 +359,7 @@ def run_ours(args, rank, world, local_rank):
     traffic = load_traffic(traffic_capture)
     recache_ms = [a.elapsed_time(b) for a, b in rev[2]]
     rc_layer_s = (sum(recache_ms) / len(recache_ms)) / 1e3 / w.layers
-    rc_flops = 2.0 * (w.slots * w.N) * w.dm * (2 * w.H * w.D)
+    rc_flops = recache_flops(w)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True,
@@ -705,7 +711,7 @@ def run_attention_only(args):
     torch.cuda.synchronize()
     times = [a.elapsed_time(b) / 1e3 for a, b in ev[args.warmup:]]
     assert swa.device_error() == 0
-    fl = 4.0 * (c * w.N) * (w.slots * w.N) * w.D * w.H
+    fl = attention_flops(w)
     peaks, kind = measured_peaks()
     t = statistics.median(times)
     return {"mode": "attention", "workload": w.name, "cache": args.cache, "launches": len(times),
@@ -823,7 +829,7 @@ def run_recache_only(args):
             times.append(a.elapsed_time(b) / 1e3)
     assert swa.device_error() == 0
     w = st.w
-    fl = 2.0 * (w.slots * w.N) * w.dm * (2 * w.H * w.D)
+    fl = recache_flops(w)
     peaks, kind = measured_peaks()
     t = statistics.median(times)
     return {"mode": "recache", "launches": len(times), "median_us": round(t * 1e6, 2),

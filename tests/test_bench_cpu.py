@@ -20,6 +20,13 @@ def test_algorithmic_flops_and_bytes():
     # append: read K, V (bf16), write them to the cache; FP8 adds one fp32 scale per (token, head)
     assert bench.append_bytes(W.WAN, 2) == 8 * n                                 # 19.2 MB
     assert bench.append_bytes(W.WAN, 1) == 4 * n + 2 * n + 2 * 1560 * 12 * 4
+    # in-place RoPE of Q: every bf16 element read once and written once
+    assert bench.rope_bytes(W.WAN, 1) == 4 * n                                   # 9.58 MB
+    assert bench.rope_bytes(W.CHUNK, 3) == 12 * n                                # 28.75 MB
+    assert round(bench.rope_bytes(W.WAN, 1) / 1e6, 2) == 9.58
+    # the recache: one GEMM of X [18720, 1536] by [Wk | Wv] [1536, 2 * 1536]
+    assert bench.recache_flops(W.STREAM) == 2 * 18720 * 1536 * 3072
+    assert round(bench.recache_flops(W.STREAM) / 1e9, 1) == 176.7
 
 
 def _sampler_with(lines):
